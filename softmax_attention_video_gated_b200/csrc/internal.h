@@ -1,0 +1,101 @@
+// internal.h -- host-side interface between the C ABI layer and the kernels.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/sva.h"
+
+namespace sva {
+
+// Launch bracketing for the stack's optional per-launch CUDA-event profile.
+struct Prof {
+  cudaEvent_t* events = nullptr;  // 2 * capacity
+  int capacity = 0;
+  int* kinds = nullptr;           // host, capacity
+  int count = 0;
+  int cur_kind = SVA_KERNEL_OTHER;
+  void before(cudaStream_t s, int kind) {
+    cur_kind = kind;
+    if (events != nullptr && count < capacity) cudaEventRecord(events[2 * count], s);
+  }
+  void after(cudaStream_t s) {
+    if (events != nullptr && count < capacity) {
+      cudaEventRecord(events[2 * count + 1], s);
+      if (kinds != nullptr) kinds[count] = cur_kind;
+    }
+    ++count;
+  }
+};
+
+struct ProfScope {
+  Prof* p;
+  cudaStream_t s;
+  ProfScope(Prof* p_, cudaStream_t s_, int kind) : p(p_), s(s_) {
+    if (p) p->before(s, kind);
+  }
+  ~ProfScope() {
+    if (p) p->after(s);
+  }
+};
+
+// ---------------------------------------------------------------- utilities
+int device_sm_count();
+int device_index();
+bool encode_tmap(CUtensorMap* map, CUtensorMapDataType dt, int rank, const void* base,
+                 const uint64_t* dims, const uint64_t* strides_bytes /* rank-1 */,
+                 const uint32_t* box, CUtensorMapSwizzle swizzle);
+
+constexpr size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+// ---------------------------------------------------------------- projections
+enum GemmEpi { EPI_STORE = 0, EPI_RESIDUAL = 1 };
+
+struct GemmArgs {
+  const void* a = nullptr;  int64_t lda = 0;   // [M, K]
+  const void* b = nullptr;  int64_t ldb = 0;   // [N, K]
+  int64_t M = 0, N = 0, K = 0;
+  int epi = EPI_STORE;
+  void* c = nullptr;        int64_t ldc = 0;   // EPI_STORE: [M, N] output
+  int relu_cols = 0;
+  float* h = nullptr;       int64_t ldh = 0;   // EPI_RESIDUAL: fp32 stream
+  void* h_copy = nullptr;   int64_t ldhc = 0;  // EPI_RESIDUAL: optional copy
+  int* status = nullptr;
+};
+
+cudaError_t gemm_bf16(const GemmArgs& g, cudaStream_t s);
+cudaError_t gemm_f32(const GemmArgs& g, cudaStream_t s);
+cudaError_t transpose_2d(const void* src, void* dst, int64_t rows, int64_t cols, sva_dtype_t dt,
+                         cudaStream_t s);  // dst[c][r] = src[r][c]
+
+// ---------------------------------------------------------------- linear attention
+// Scratch of one linear-attention call (offsets from the scratch base):
+// fp32 per-chunk partial states, then the reduced state.
+struct LinearPlan {
+  int tiles_per_chunk = 0;  // 128-token tiles per state chunk (bf16) / tokens per chunk (f32)
+  int n_chunks = 0;
+  size_t partial_off = 0, state_off = 0, total = 0;
+};
+LinearPlan linear_plan(int B, int N, int H, int d, sva_dtype_t dt);
+cudaError_t linear_bf16(const sva_attn_args& a, int* status, void* scratch, cudaStream_t s,
+                        Prof* prof);
+cudaError_t linear_f32(const sva_attn_args& a, int* status, void* scratch, cudaStream_t s,
+                       Prof* prof);
+
+// ---------------------------------------------------------------- softmax anchor
+cudaError_t anchor_bf16(const sva_attn_args& a, int* status, cudaStream_t s);
+cudaError_t anchor_f32(const sva_attn_args& a, int* status, cudaStream_t s);
+
+// ---------------------------------------------------------------- router
+cudaError_t route(const float* h, const void* const* keys, const void* const* summaries,
+                  int n_blocks, void* u, float* alpha, int64_t rows, int D, sva_dtype_t dt,
+                  cudaStream_t s);
+
+// ---------------------------------------------------------------- misc
+cudaError_t selftest_wait(int* status, unsigned timeout_us, cudaStream_t s);
+cudaError_t cast_f32(const float* src, void* dst, int64_t n, sva_dtype_t dt, cudaStream_t s);
+cudaError_t upcast_to_f32(const void* src, float* dst, int64_t n, sva_dtype_t dt, cudaStream_t s);
+cudaError_t sub_inplace(const float* a, float* out, int64_t n, cudaStream_t s);  // out = a - out
+
+}  // namespace sva

@@ -1,0 +1,544 @@
+// linear_tc.cu -- gated linear attention, bf16, d = 128, on tcgen05/TMEM.
+//
+// The layer keeps a fixed-size state per (batch, head) and costs O(N)
+// [ai-papers.net summary, section "ハイブリッド線形アテンション"]. With phi = ReLU:
+//   S = sum_t phi(K_t)^T V_t,  z = sum_t phi(K_t),
+//   Y_t = phi(Q_t) S / (phi(Q_t) . z + eps) * sigmoid(G_t)   (+ residual).
+//
+// Three kernels, all HBM-bound (the roofline is 10 B*N*D bytes of Q, K, V, G
+// and Y traffic per layer):
+//  1. lin_state_tc:  one CTA per (token chunk, head, batch). TMA streams
+//     128-token K and V tiles into a 3-stage ring; four warps apply ReLU in
+//     shared memory and accumulate z; one thread issues tcgen05.mma with
+//     A = phi(K)^T and B = V, both read MN-major straight from the TMA layout,
+//     accumulating the 128x128 fp32 partial state in TMEM.
+//  2. lin_reduce: sums the chunk partials in chunk order (deterministic) and
+//     writes the read-out operand [S^T | z_hi | z_lo | 0] as bf16 [144 x 128]
+//     (z split in two bf16 rows keeps it to ~16 bits).
+//  3. lin_readout_tc: one CTA per 128-token tile. TMA loads Q, G and the
+//     state operand; ReLU on Q in shared memory; one M=128, N=144, K=128 MMA
+//     gives the numerator (columns 0..127) and denominator (columns 128, 129)
+//     together; the epilogue divides, applies the sigmoid gate and residual,
+//     and writes Y through a TMA store.
+#include <algorithm>
+
+#include "common.cuh"
+#include "internal.h"
+
+namespace sva {
+namespace {
+
+constexpr int HD = 128;                 // head dim of these kernels
+constexpr int TT = 128;                 // tokens per tile
+constexpr int BOX_BYTES = TT * 128;     // one [64 cols x 128 rows] bf16 box = 16 KB
+constexpr int STATE_ROWS = HD + 16;     // read-out B operand rows: S^T, z_hi, z_lo, zeros
+constexpr int STATE_BOX_BYTES = STATE_ROWS * 128;
+
+// ------------------------------------------------------------------ state
+constexpr int ST_STAGES = 3;
+constexpr int ST_STAGE_BYTES = 4 * BOX_BYTES;  // K (2 boxes) + V (2 boxes)
+
+struct StateTail {
+  uint64_t full[ST_STAGES];
+  uint64_t relu_done[ST_STAGES];
+  uint64_t empty[ST_STAGES];
+  uint64_t s_full;
+  uint64_t drain;
+  uint32_t tmem_base;
+  int abort_flag;
+  float zbuf[8][HD];
+};
+constexpr size_t kStateSmem = 1024 + ST_STAGES * ST_STAGE_BYTES + sizeof(StateTail);
+
+__device__ __forceinline__ bool drain_wait(uint64_t* bar, uint32_t parity) {
+  int never = 0;
+  return mbar_wait(bar, parity, &never, nullptr, 0);
+}
+
+__global__ void __launch_bounds__(192, 1)
+    lin_state_tc_kernel(const __grid_constant__ CUtensorMap map_k,
+                        const __grid_constant__ CUtensorMap map_v, int N, int H,
+                        int tiles_per_chunk, int n_chunks, unsigned flags, float* partial,
+                        int* status) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  StateTail* tl = reinterpret_cast<StateTail*>(smem + ST_STAGES * ST_STAGE_BYTES);
+  const int c = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+  const int warp = warp_id(), lane = lane_id();
+  const int tiles_total = (N + TT - 1) / TT;
+  const int tile0 = c * tiles_per_chunk;
+  const int ntiles = max(0, min(tiles_per_chunk, tiles_total - tile0));
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < ST_STAGES; ++s) {
+      mbar_init(&tl->full[s], 1);
+      mbar_init(&tl->relu_done[s], 128);
+      mbar_init(&tl->empty[s], 1);
+    }
+    mbar_init(&tl->s_full, 1);
+    mbar_init(&tl->drain, 1);
+    tl->abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(&tl->tmem_base, HD);
+    tmem_relinquish();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&map_k);
+    tma_prefetch_desc(&map_v);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = tl->tmem_base;
+  volatile int* abort_flag = &tl->abort_flag;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      int issued = 0;
+      bool ok = true;
+      for (int i = 0; i < ntiles; ++i) {
+        if (!mbar_wait(&tl->empty[stage], phase ^ 1, abort_flag, status, WHERE_LIN_STATE)) {
+          ok = false;
+          break;
+        }
+        uint8_t* st = smem + stage * ST_STAGE_BYTES;
+        const int t0 = (tile0 + i) * TT;
+        mbar_arrive_expect_tx(&tl->full[stage], ST_STAGE_BYTES);
+        tma_load_3d(&map_k, &tl->full[stage], st, h * HD, t0, b);
+        tma_load_3d(&map_k, &tl->full[stage], st + BOX_BYTES, h * HD + 64, t0, b);
+        tma_load_3d(&map_v, &tl->full[stage], st + 2 * BOX_BYTES, h * HD, t0, b);
+        tma_load_3d(&map_v, &tl->full[stage], st + 3 * BOX_BYTES, h * HD + 64, t0, b);
+        ++issued;
+        if (++stage == ST_STAGES) {
+          stage = 0;
+          phase ^= 1;
+        }
+      }
+      if (!ok)
+        for (int i = max(0, issued - ST_STAGES); i < issued; ++i)
+          (void)drain_wait(&tl->full[i % ST_STAGES], (i / ST_STAGES) & 1);
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      // A = phi(K)^T: M = d (MN-major, the 64-wide d atoms 16 KB apart),
+      // B = V: N = d (MN-major), K = tokens (8-token groups 1024 B apart).
+      constexpr uint32_t idesc = idesc_bf16_f32(HD, HD, true, true);
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      for (int i = 0; i < ntiles; ++i) {
+        if (!mbar_wait(&tl->relu_done[stage], phase, abort_flag, status, WHERE_LIN_STATE)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t kaddr = smem_u32(smem + stage * ST_STAGE_BYTES);
+        const uint32_t vaddr = kaddr + 2 * BOX_BYTES;
+#pragma unroll
+        for (int kk = 0; kk < TT / 16; ++kk) {
+          const uint64_t ad = smem_desc(kaddr + kk * 2048, BOX_BYTES, 1024);
+          const uint64_t bd = smem_desc(vaddr + kk * 2048, BOX_BYTES, 1024);
+          umma_ss(tmem, ad, bd, idesc, (i | kk) != 0 ? 1u : 0u);
+        }
+        umma_commit(&tl->empty[stage]);
+        if (++stage == ST_STAGES) {
+          stage = 0;
+          phase ^= 1;
+        }
+      }
+      if (ok) umma_commit(&tl->s_full);
+      umma_commit(&tl->drain);
+      (void)drain_wait(&tl->drain, 0);
+    }
+  } else {
+    // ---------------------------------------- ReLU + z workers, then epilogue
+    const int wt = threadIdx.x - 64;          // 0..127
+    const int ch = wt & 15;                   // logical 16-byte chunk of a row (8 columns)
+    const int rc = wt >> 4;                   // row class: rows rc, rc+8, ...
+    const int box = ch >> 3, cl = ch & 7;
+    const uint32_t col_off = box * BOX_BYTES + ((cl ^ rc) << 4);
+    const bool features = (flags & SVA_FLAG_QK_FEATURES) != 0;
+    float z[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) z[i] = 0.f;
+    int stage = 0;
+    uint32_t phase = 0;
+    bool ok = true;
+    for (int i = 0; i < ntiles; ++i) {
+      bool w = mbar_wait(&tl->full[stage], phase, abort_flag, status, WHERE_LIN_STATE);
+      if (!__all_sync(0xffffffffu, w)) {
+        ok = false;
+        break;
+      }
+      uint8_t* kt = smem + stage * ST_STAGE_BYTES + col_off;
+#pragma unroll 4
+      for (int j = 0; j < TT / 8; ++j) {
+        uint4* p = reinterpret_cast<uint4*>(kt + (rc + 8 * j) * 128);
+        uint4 v = *p;
+        if (!features) {
+          v.x = relu_bf16x2(v.x);
+          v.y = relu_bf16x2(v.y);
+          v.z = relu_bf16x2(v.z);
+          v.w = relu_bf16x2(v.w);
+          *p = v;
+        }
+        z[0] += bf16lo_to_f32(v.x); z[1] += bf16hi_to_f32(v.x);
+        z[2] += bf16lo_to_f32(v.y); z[3] += bf16hi_to_f32(v.y);
+        z[4] += bf16lo_to_f32(v.z); z[5] += bf16hi_to_f32(v.z);
+        z[6] += bf16lo_to_f32(v.w); z[7] += bf16hi_to_f32(v.w);
+      }
+      fence_proxy_async_smem();
+      mbar_arrive(&tl->relu_done[stage]);
+      if (++stage == ST_STAGES) {
+        stage = 0;
+        phase ^= 1;
+      }
+    }
+    // z: reduce the 8 row classes
+#pragma unroll
+    for (int i = 0; i < 8; ++i) tl->zbuf[rc][ch * 8 + i] = z[i];
+    named_barrier_sync(1, 128);
+    float* out = partial + (static_cast<int64_t>(b * H + h) * n_chunks + c) * (HD * HD + HD);
+    {
+      float zs = 0.f;
+#pragma unroll
+      for (int r = 0; r < 8; ++r) zs += tl->zbuf[r][wt];
+      out[HD * HD + wt] = zs;
+    }
+    // partial state rows: TMEM lane = d_k index, column = d_v index
+    const int q = warp & 3;
+    const int row = q * 32 + lane;
+    bool have = ok && ntiles > 0;
+    if (have) {
+      bool w = mbar_wait(&tl->s_full, 0, abort_flag, status, WHERE_LIN_STATE);
+      have = __all_sync(0xffffffffu, w);
+    }
+    if (have) {
+      tc_fence_after();
+#pragma unroll 1
+      for (int cc = 0; cc < HD; cc += 32) {
+        uint32_t r[32];
+        tmem_ld32(tmem + (static_cast<uint32_t>(q * 32) << 16) + cc, r);
+        tmem_wait_ld();
+        float4* dst = reinterpret_cast<float4*>(out + row * HD + cc);
+#pragma unroll
+        for (int k = 0; k < 8; ++k)
+          dst[k] = make_float4(__uint_as_float(r[4 * k]), __uint_as_float(r[4 * k + 1]),
+                               __uint_as_float(r[4 * k + 2]), __uint_as_float(r[4 * k + 3]));
+      }
+    } else if (ntiles == 0) {
+      float4* dst = reinterpret_cast<float4*>(out + row * HD);
+      for (int k = 0; k < HD / 4; ++k) dst[k] = make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, HD);
+  }
+}
+
+// ------------------------------------------------------------------ reduce
+// state_op[bh] = bf16 [144][128]: rows 0..127 = S^T (row n = d_v, column k =
+// d_k), row 128 = bf16(z), row 129 = bf16(z - bf16(z)), rows 130..143 = 0.
+__global__ void __launch_bounds__(256) lin_reduce_bf16_kernel(const float* __restrict__ partial,
+                                                              __nv_bfloat16* __restrict__ state_op,
+                                                              int n_chunks) {
+  const int64_t bh = blockIdx.x;
+  const int elems = HD * HD + HD;
+  const float* p = partial + bh * n_chunks * elems;
+  __nv_bfloat16* o = state_op + bh * STATE_ROWS * HD;
+  for (int e = threadIdx.x; e < HD * HD; e += 256) {
+    float s = 0.f;
+    for (int c = 0; c < n_chunks; ++c) s += p[static_cast<int64_t>(c) * elems + e];
+    const int k = e / HD, n = e % HD;
+    o[n * HD + k] = __float2bfloat16_rn(s);
+  }
+  for (int e = threadIdx.x; e < HD; e += 256) {
+    float s = 0.f;
+    for (int c = 0; c < n_chunks; ++c) s += p[static_cast<int64_t>(c) * elems + HD * HD + e];
+    const __nv_bfloat16 hi = __float2bfloat16_rn(s);
+    o[HD * HD + e] = hi;
+    o[(HD + 1) * HD + e] = __float2bfloat16_rn(s - __bfloat162float(hi));
+  }
+  for (int e = threadIdx.x; e < (STATE_ROWS - HD - 2) * HD; e += 256)
+    o[(HD + 2) * HD + e] = __float2bfloat16_rn(0.f);
+}
+
+// ------------------------------------------------------------------ read-out
+struct ReadoutTail {
+  uint64_t full_qs;
+  uint64_t full_g;
+  uint64_t relu_done;
+  uint64_t acc_full;
+  uint64_t drain;
+  uint32_t tmem_base;
+  int abort_flag;
+};
+constexpr int RO_Q_OFF = 0;                                   // 32 KB, reused for Y
+constexpr int RO_G_OFF = 2 * BOX_BYTES;                       // 32 KB
+constexpr int RO_S_OFF = 4 * BOX_BYTES;                       // 36 KB
+constexpr int RO_TAIL_OFF = RO_S_OFF + 2 * STATE_BOX_BYTES;
+constexpr size_t kReadoutSmem = 1024 + RO_TAIL_OFF + sizeof(ReadoutTail);
+constexpr int RO_TMEM_COLS = 256;
+
+__global__ void __launch_bounds__(192)
+    lin_readout_tc_kernel(const __grid_constant__ CUtensorMap map_q,
+                          const __grid_constant__ CUtensorMap map_g,
+                          const __grid_constant__ CUtensorMap map_s,
+                          const __grid_constant__ CUtensorMap map_o, int N, int H, float eps,
+                          unsigned flags, const __nv_bfloat16* residual, int64_t ldr,
+                          int* status) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  ReadoutTail* tl = reinterpret_cast<ReadoutTail*>(smem + RO_TAIL_OFF);
+  const int tile = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+  const int t0 = tile * TT;
+  const int warp = warp_id(), lane = lane_id();
+
+  if (threadIdx.x == 0) {
+    mbar_init(&tl->full_qs, 1);
+    mbar_init(&tl->full_g, 1);
+    mbar_init(&tl->relu_done, 128);
+    mbar_init(&tl->acc_full, 1);
+    mbar_init(&tl->drain, 1);
+    tl->abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(&tl->tmem_base, RO_TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = tl->tmem_base;
+  volatile int* abort_flag = &tl->abort_flag;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      const int srow = (b * H + h) * STATE_ROWS;
+      mbar_arrive_expect_tx(&tl->full_qs, 2 * BOX_BYTES + 2 * STATE_BOX_BYTES);
+      tma_load_3d(&map_q, &tl->full_qs, smem + RO_Q_OFF, h * HD, t0, b);
+      tma_load_3d(&map_q, &tl->full_qs, smem + RO_Q_OFF + BOX_BYTES, h * HD + 64, t0, b);
+      tma_load_2d(&map_s, &tl->full_qs, smem + RO_S_OFF, 0, srow);
+      tma_load_2d(&map_s, &tl->full_qs, smem + RO_S_OFF + STATE_BOX_BYTES, 64, srow);
+      mbar_arrive_expect_tx(&tl->full_g, 2 * BOX_BYTES);
+      tma_load_3d(&map_g, &tl->full_g, smem + RO_G_OFF, h * HD, t0, b);
+      tma_load_3d(&map_g, &tl->full_g, smem + RO_G_OFF + BOX_BYTES, h * HD + 64, t0, b);
+      // both barriers are waited on below by the epilogue threads before exit,
+      // (bounded), so no load is left in flight when the CTA finishes
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      constexpr uint32_t idesc = idesc_bf16_f32(128, STATE_ROWS, false, false);
+      if (mbar_wait(&tl->relu_done, 0, abort_flag, status, WHERE_LIN_READOUT)) {
+        tc_fence_after();
+        const uint32_t qaddr = smem_u32(smem + RO_Q_OFF);
+        const uint32_t saddr = smem_u32(smem + RO_S_OFF);
+#pragma unroll
+        for (int kk = 0; kk < HD / 16; ++kk) {
+          const int bx = kk >> 2, w = kk & 3;
+          const uint64_t ad = smem_desc(qaddr + bx * BOX_BYTES + w * 32, 16, 1024);
+          const uint64_t bd = smem_desc(saddr + bx * STATE_BOX_BYTES + w * 32, 16, 1024);
+          umma_ss(tmem, ad, bd, idesc, kk != 0 ? 1u : 0u);
+        }
+        umma_commit(&tl->acc_full);
+      }
+      umma_commit(&tl->drain);
+      (void)drain_wait(&tl->drain, 0);
+    }
+  } else {
+    const int wt = threadIdx.x - 64;
+    const int q = warp & 3;
+    bool ok;
+    {
+      // ReLU on the Q tile, in place
+      bool w = mbar_wait(&tl->full_qs, 0, abort_flag, status, WHERE_LIN_READOUT);
+      ok = __all_sync(0xffffffffu, w);
+      if (ok && (flags & SVA_FLAG_QK_FEATURES) == 0) {
+        const int ch = wt & 15, rc = wt >> 4;
+        const int box = ch >> 3, cl = ch & 7;
+        uint8_t* qt = smem + RO_Q_OFF + box * BOX_BYTES + ((cl ^ rc) << 4);
+#pragma unroll 4
+        for (int j = 0; j < TT / 8; ++j) {
+          uint4* p = reinterpret_cast<uint4*>(qt + (rc + 8 * j) * 128);
+          uint4 v = *p;
+          v.x = relu_bf16x2(v.x);
+          v.y = relu_bf16x2(v.y);
+          v.z = relu_bf16x2(v.z);
+          v.w = relu_bf16x2(v.w);
+          *p = v;
+        }
+        fence_proxy_async_smem();
+      }
+      if (ok) mbar_arrive(&tl->relu_done);
+    }
+    if (ok) {
+      bool w = mbar_wait(&tl->acc_full, 0, abort_flag, status, WHERE_LIN_READOUT);
+      w = w && mbar_wait(&tl->full_g, 0, abort_flag, status, WHERE_LIN_READOUT);
+      ok = __all_sync(0xffffffffu, w);
+    }
+    if (ok) {
+      tc_fence_after();
+      const int r = q * 32 + lane;                 // row of the tile = TMEM lane
+      const uint32_t trow = tmem + (static_cast<uint32_t>(q * 32) << 16);
+      uint32_t dd[16];
+      tmem_ld16(trow + HD, dd);
+      tmem_wait_ld();
+      const float inv = 1.0f / (__uint_as_float(dd[0]) + __uint_as_float(dd[1]) + eps);
+      const int t = t0 + r;
+      const bool row_ok = t < N;
+      const __nv_bfloat16* res =
+          (residual != nullptr && row_ok)
+              ? residual + (static_cast<int64_t>(b) * N + t) * ldr + h * HD
+              : nullptr;
+#pragma unroll 1
+      for (int cc = 0; cc < HD; cc += 32) {
+        uint32_t num[32];
+        tmem_ld32(trow + cc, num);
+        tmem_wait_ld();
+        const int box = cc >> 6;
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const int cl = ((cc & 63) >> 3) + k;
+          const uint32_t off = box * BOX_BYTES + r * 128 + ((cl ^ (r & 7)) << 4);
+          const uint4 gv = *reinterpret_cast<const uint4*>(smem + RO_G_OFF + off);
+          float gg[8] = {bf16lo_to_f32(gv.x), bf16hi_to_f32(gv.x), bf16lo_to_f32(gv.y),
+                         bf16hi_to_f32(gv.y), bf16lo_to_f32(gv.z), bf16hi_to_f32(gv.z),
+                         bf16lo_to_f32(gv.w), bf16hi_to_f32(gv.w)};
+          float y[8];
+#pragma unroll
+          for (int e = 0; e < 8; ++e)
+            y[e] = __uint_as_float(num[8 * k + e]) * inv * fast_sigmoid(gg[e]);
+          if (res != nullptr) {
+            const uint4 rv = *reinterpret_cast<const uint4*>(res + cc + 8 * k);
+            y[0] += bf16lo_to_f32(rv.x); y[1] += bf16hi_to_f32(rv.x);
+            y[2] += bf16lo_to_f32(rv.y); y[3] += bf16hi_to_f32(rv.y);
+            y[4] += bf16lo_to_f32(rv.z); y[5] += bf16hi_to_f32(rv.z);
+            y[6] += bf16lo_to_f32(rv.w); y[7] += bf16hi_to_f32(rv.w);
+          }
+          uint4 o;
+          o.x = pack_bf16x2(y[0], y[1]);
+          o.y = pack_bf16x2(y[2], y[3]);
+          o.z = pack_bf16x2(y[4], y[5]);
+          o.w = pack_bf16x2(y[6], y[7]);
+          *reinterpret_cast<uint4*>(smem + RO_Q_OFF + off) = o;
+        }
+      }
+      fence_proxy_async_smem();
+    } else {
+      // make sure no TMA load is still writing shared memory before exit
+      (void)drain_wait(&tl->full_qs, 0);
+      (void)drain_wait(&tl->full_g, 0);
+    }
+    named_barrier_sync(1, 128);
+    if (ok && wt == 0) {
+      tma_store_3d(&map_o, smem + RO_Q_OFF, h * HD, t0, b);
+      tma_store_3d(&map_o, smem + RO_Q_OFF + BOX_BYTES, h * HD + 64, t0, b);
+      tma_store_commit();
+      tma_store_wait_read0();
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, RO_TMEM_COLS);
+  }
+}
+
+bool act_map(CUtensorMap* m, const void* base, int64_t ld, int B, int N, int D) {
+  const uint64_t dims[3] = {static_cast<uint64_t>(D), static_cast<uint64_t>(N),
+                            static_cast<uint64_t>(B)};
+  const uint64_t strides[2] = {static_cast<uint64_t>(ld) * 2,
+                               static_cast<uint64_t>(ld) * 2 * static_cast<uint64_t>(N)};
+  const uint32_t box[3] = {64, TT, 1};
+  return encode_tmap(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, base, dims, strides, box,
+                     CU_TENSOR_MAP_SWIZZLE_128B);
+}
+
+}  // namespace
+
+LinearPlan linear_plan(int B, int N, int H, int d, sva_dtype_t dt) {
+  LinearPlan p;
+  const int64_t work = static_cast<int64_t>(B) * H;
+  const int sms = std::max(1, device_sm_count());
+  if (dt == SVA_BF16) {
+    // one wave: the fewest tiles per chunk with work * n_chunks <= #SMs
+    const int tiles = (N + TT - 1) / TT;
+    int ct = 1;
+    while (ct < tiles && work * ((tiles + ct - 1) / ct) > sms) ++ct;
+    p.tiles_per_chunk = ct;
+    p.n_chunks = (tiles + ct - 1) / ct;
+  } else {
+    const int tokens = 256;
+    p.tiles_per_chunk = tokens;
+    p.n_chunks = (N + tokens - 1) / tokens;
+  }
+  const size_t elems = static_cast<size_t>(d) * d + d;
+  p.partial_off = 0;
+  p.state_off = align_up(p.partial_off + static_cast<size_t>(p.n_chunks) * work * elems * 4, 1024);
+  const size_t state_bytes = dt == SVA_BF16 ? static_cast<size_t>(work) * STATE_ROWS * HD * 2
+                                            : static_cast<size_t>(work) * elems * 4;
+  p.total = align_up(p.state_off + state_bytes, 1024);
+  return p;
+}
+
+cudaError_t linear_bf16(const sva_attn_args& a, int* status, void* scratch, cudaStream_t s,
+                        Prof* prof) {
+  const LinearPlan p = linear_plan(a.B, a.N, a.H, a.d, SVA_BF16);
+  char* base = static_cast<char*>(scratch);
+  float* partial = reinterpret_cast<float*>(base + p.partial_off);
+  __nv_bfloat16* state = reinterpret_cast<__nv_bfloat16*>(base + p.state_off);
+  const int D = a.H * a.d;
+  CUtensorMap mk, mv, mq, mg, mo, ms;
+  if (!act_map(&mk, a.k, a.ldk, a.B, a.N, D) || !act_map(&mv, a.v, a.ldv, a.B, a.N, D) ||
+      !act_map(&mq, a.q, a.ldq, a.B, a.N, D) || !act_map(&mg, a.gate, a.ldg, a.B, a.N, D) ||
+      !act_map(&mo, a.out, a.ldo, a.B, a.N, D))
+    return cudaErrorInvalidValue;
+  {
+    const uint64_t dims[2] = {HD, static_cast<uint64_t>(a.B) * a.H * STATE_ROWS};
+    const uint64_t strides[1] = {HD * 2};
+    const uint32_t box[2] = {64, STATE_ROWS};
+    if (!encode_tmap(&ms, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, state, dims, strides, box,
+                     CU_TENSOR_MAP_SWIZZLE_128B))
+      return cudaErrorInvalidValue;
+  }
+  cudaError_t e;
+  {
+    ProfScope ps(prof, s, SVA_KERNEL_LINEAR_STATE);
+    e = cudaFuncSetAttribute(lin_state_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(kStateSmem));
+    if (e != cudaSuccess) return e;
+    dim3 grid(p.n_chunks, a.H, a.B);
+    lin_state_tc_kernel<<<grid, 192, kStateSmem, s>>>(mk, mv, a.N, a.H, p.tiles_per_chunk,
+                                                      p.n_chunks, a.flags, partial, status);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  }
+  {
+    ProfScope ps(prof, s, SVA_KERNEL_LINEAR_STATE);
+    lin_reduce_bf16_kernel<<<a.B * a.H, 256, 0, s>>>(partial, state, p.n_chunks);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  }
+  ProfScope ps(prof, s, SVA_KERNEL_LINEAR_READOUT);
+  e = cudaFuncSetAttribute(lin_readout_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           static_cast<int>(kReadoutSmem));
+  if (e != cudaSuccess) return e;
+  dim3 grid((a.N + TT - 1) / TT, a.H, a.B);
+  lin_readout_tc_kernel<<<grid, 192, kReadoutSmem, s>>>(
+      mq, mg, ms, mo, a.N, a.H, a.eps, a.flags, static_cast<const __nv_bfloat16*>(a.residual),
+      a.ldr, status);
+  return cudaGetLastError();
+}
+
+}  // namespace sva

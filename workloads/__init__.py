@@ -174,3 +174,22 @@ def stack_weights(w: StackWorkload, layers: Optional[Sequence[int]] = None,
 
 def stack_x(w: StackWorkload) -> np.ndarray:
     return normal((w.B, w.N, w.D), 1.0, w.seed, TAG_X, w.dtype)
+
+
+# ---------------------------------------------------------------------------
+# device-side draws for bench-size tensors
+# ---------------------------------------------------------------------------
+
+
+def normal_torch(shape, std: float, seed: int, tag: int, dtype: str, device="cuda"):
+    """N(0, std^2) drawn by torch's seeded Philox generator on `device`, rounded
+    to `dtype` (torch's round-to-nearest-even). Used where numpy would take
+    minutes (the 720p stack's 1.1e9 weights); tensors drawn here are never
+    compared element by element with the oracle."""
+    import torch
+    g = torch.Generator(device=device)
+    g.manual_seed((seed * 1000003 + tag) & 0x7FFFFFFFFFFFFFFF)
+    t = torch.randn(shape, generator=g, device=device, dtype=torch.float32)
+    if std != 1.0:
+        t.mul_(std)
+    return t.to(torch.bfloat16) if dtype == "bf16" else t

@@ -97,6 +97,22 @@ sva_status_t sva_linear_attn_fwd(const sva_attn_args* args, void* ws, size_t ws_
                                  sva_stream_t stream);
 
 /*
+ * Allocation-free variant of sva_linear_attn_fwd (same arguments, same
+ * results) for callers that cannot allocate device memory when they run the
+ * mixer: engines that plan all device memory at start-up and allow no
+ * allocation afterwards, plugins handed a stream but no allocator, programs
+ * whose memory pool belongs to another framework. The paper has no
+ * counterpart; this is a library convenience. The scratch is a 16 MiB
+ * file-scope device array held by every GPU that loads the library until
+ * exit; calls needing more return SVA_ERR_WORKSPACE before launching
+ * anything. The first call on a device looks up the array's address (make it
+ * before any stream capture). All calls on a device share the array: calls
+ * that overlap on the GPU race and must be serialised by the caller.
+ * Device-side timeouts are not reported by this entry point.
+ */
+sva_status_t sva_linear_attn_fwd_noalloc(const sva_attn_args* args, sva_stream_t stream);
+
+/*
  * Gated softmax anchor (non-causal), every fourth layer of the hybrid
  * [lode.cx summary, "How It Works": gated softmax keeps exact token relations;
  * SANA-Video 2.0 abstract: periodic gated-softmax anchors at a 3:1 ratio]:

@@ -71,6 +71,7 @@ _SIGS = {
     "sva_linear_attn_workspace_bytes": (ctypes.c_size_t, [ctypes.c_int] * 4 + [ctypes.c_int]),
     "sva_linear_attn_fwd": (ctypes.c_int, [ctypes.POINTER(AttnArgs), ctypes.c_void_p,
                                            ctypes.c_size_t, ctypes.c_void_p]),
+    "sva_linear_attn_fwd_noalloc": (ctypes.c_int, [ctypes.POINTER(AttnArgs), ctypes.c_void_p]),
     "sva_softmax_anchor_workspace_bytes": (ctypes.c_size_t, [ctypes.c_int] * 5),
     "sva_softmax_anchor_fwd": (ctypes.c_int, [ctypes.POINTER(AttnArgs), ctypes.c_void_p,
                                               ctypes.c_size_t, ctypes.c_void_p]),
@@ -221,6 +222,16 @@ def sva_linear_attn_fwd(q, k, v, gate, out, H: int, residual=None, eps: float = 
     _check(_lib().sva_linear_attn_fwd(ctypes.byref(a), _ptr(ws), ws.numel(), _stream(stream)),
            "sva_linear_attn_fwd")
     return ws
+
+
+def sva_linear_attn_fwd_noalloc(q, k, v, gate, out, H: int, residual=None, eps: float = 1e-6,
+                                flags: int = 0, stream=None):
+    """sva_linear_attn_fwd without a workspace, for callers that cannot allocate
+    device memory: the library's fixed 16 MiB device scratch is used instead.
+    Calls that overlap on the GPU share that scratch and must be serialised."""
+    a = _attn_args(q, k, v, gate, out, H, residual, eps, 0.0, flags)
+    _check(_lib().sva_linear_attn_fwd_noalloc(ctypes.byref(a), _stream(stream)),
+           "sva_linear_attn_fwd_noalloc")
 
 
 def sva_softmax_anchor_fwd(q, k, v, gate, out, H: int, residual=None, scale: float = 0.0,

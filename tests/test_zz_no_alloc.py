@@ -1,0 +1,51 @@
+"""The allocation-free linear-attention entry point, for callers that cannot
+allocate device memory (an engine with a fixed memory plan, a plugin handed a
+stream but no allocator): it must give the same results as the workspace entry
+point, call after call, while its scratch lives in the library's fixed device
+array. Collected last so a failure here leaves every other test already run."""
+import ctypes
+
+import numpy as np
+import pytest
+
+import workloads as W
+from tests._util import assert_close, to_dev, to_host
+
+pytestmark = pytest.mark.gpu
+
+torch = pytest.importorskip("torch")
+if not torch.cuda.is_available():
+    pytest.skip("needs a CUDA device", allow_module_level=True)
+
+import softmax_attention_video_gated_b200 as sva  # noqa: E402
+
+
+def noalloc_call(q, k, v, g, out, H, eps=1e-6):
+    a = sva._attn_args(q, k, v, g, out, H, None, eps, 0.0, 0)
+    return sva._lib().sva_linear_attn_fwd_noalloc(ctypes.byref(a), sva._stream())
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_noalloc_matches_workspace_entry_point_on_two_calls_in_a_row(dtype):
+    # two calls with different shapes and values: the second must not see the
+    # first one's scratch
+    for B, N, H, seed in ((2, 1000, 2, 101), (1, 3001, 3, 102)):
+        x = W.core_inputs(B, N, H, 128, dtype, seed)
+        t = {k: to_dev(v, dtype) for k, v in x.items()}
+        ref = torch.empty_like(t["q"])
+        sva.sva_linear_attn_fwd(t["q"], t["k"], t["v"], t["g"], ref, H, eps=1e-6)
+        out = torch.full_like(t["q"], float("nan"))
+        assert noalloc_call(t["q"], t["k"], t["v"], t["g"], out, H) == sva.SVA_OK
+        torch.cuda.synchronize()
+        assert_close(to_host(out), to_host(ref), dtype, f"noalloc B={B} N={N}")
+
+
+def test_noalloc_refuses_calls_beyond_its_scratch():
+    # fp32, 128 heads of d = 128 over 100k tokens needs far more than 16 MiB
+    a = sva.AttnArgs()
+    a.B, a.N, a.H, a.d, a.dtype = 1, 100000, 128, 128, sva.SVA_F32
+    for f in ("q", "k", "v", "gate", "out"):
+        setattr(a, f, 0x10000)
+    a.ldq = a.ldk = a.ldv = a.ldg = a.ldo = 128 * 128
+    a.eps = 1e-6
+    assert sva._lib().sva_linear_attn_fwd_noalloc(ctypes.byref(a), None) == sva.SVA_ERR_WORKSPACE

@@ -41,7 +41,7 @@ WORKLOAD = dict(name="720p-shaped 24-layer hybrid stack (18 gated linear + 6 gat
                 B=1, N=19320, H=24, d=128, L=24, softmax_period=4, attnres_block=8)
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 KINDS = ("proj_qkvg", "proj_out", "linear_state", "linear_readout", "anchor", "route", "keys",
-         "other")
+         "other", "linear_reduce")
 
 
 # ---------------------------------------------------------------------------
@@ -340,6 +340,58 @@ def summarize(recs, steps, wl, peaks):
     return out
 
 
+def run_case(args):
+    """One kernel class on its own (for sweeps and profiler captures): prints a
+    JSON line with the device time per launch and the achieved rate."""
+    import torch
+
+    import softmax_attention_video_gated_b200 as sva
+    import workloads as W
+
+    peaks = load_peaks()
+    B, N, H, d = args.B, args.N, args.H, 128
+    D = H * d
+    seed = 77
+    if args.case in ("anchor", "linear"):
+        q, k, v, g = (W.normal_torch((B, N, D), 1.0, seed, tag, "bf16")
+                      for tag in (W.TAG_Q, W.TAG_K, W.TAG_V, W.TAG_G))
+        out = torch.empty_like(q)
+        if args.case == "anchor":
+            ws = sva.workspace(256)
+            fn = lambda: sva.sva_softmax_anchor_fwd(q, k, v, g, out, H, ws=ws)  # noqa: E731
+            work, unit = 4.0 * B * N * N * D, "TFLOP/s"
+        else:
+            ws = sva.workspace(sva.sva_linear_attn_workspace_bytes(B, N, H, d, sva.SVA_BF16))
+            fn = lambda: sva.sva_linear_attn_fwd(q, k, v, g, out, H, ws=ws)  # noqa: E731
+            work, unit = 10.0 * B * N * D, "GB/s"
+    else:
+        M, K, Nout = B * N, D, 4 * D
+        x = W.normal_torch((M, K), 1.0, seed, W.TAG_X, "bf16")
+        w = W.normal_torch((Nout, K), 1.0 / math.sqrt(K), seed, W.TAG_WQKVG, "bf16")
+        y = torch.empty(M, Nout, device="cuda", dtype=torch.bfloat16)
+        ws = sva.workspace(256)
+        fn = lambda: sva.sva_projection_fwd(x, w, y, ws=ws)  # noqa: E731
+        work, unit = 2.0 * M * K * Nout, "TFLOP/s"
+    for _ in range(args.warmup):
+        fn()
+    torch.cuda.synchronize()
+    st = sva.sva_check_device_status(ws)
+    if st != sva.SVA_OK:
+        raise RuntimeError(sva.status_string(st))
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(args.steps):
+        fn()
+    e1.record()
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / args.steps
+    rate = work / (ms * 1e-3) / (1e12 if unit == "TFLOP/s" else 1e9)
+    peak = peaks["bf16_tflops"] if unit == "TFLOP/s" else peaks["hbm_gbs"]
+    print(json.dumps({"case": args.case, "B": B, "N": N, "H": H, "ms_per_launch": ms,
+                      "achieved": rate, "unit": unit, "frac_of_burst_peak": rate / peak}), flush=True)
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
@@ -348,10 +400,17 @@ def main():
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-all-softmax", action="store_true")
+    ap.add_argument("--case", choices=("anchor", "linear", "gemm"),
+                    help="time one kernel class alone instead of the stack")
+    ap.add_argument("--B", type=int, default=1)
+    ap.add_argument("--N", type=int, default=19320)
+    ap.add_argument("--H", type=int, default=24)
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
     wl = dict(WORKLOAD)
+    if args.case:
+        return run_case(args)
     if args.impl == "reference":
         return run_reference(args, wl)
 
@@ -457,7 +516,8 @@ def main():
         sva.sva_hybrid_stack_fwd(st_all, x, y, ws_all)
         ms_all, recs_all, _ = timed_steps(torch, sva, st_all, x, y, ws_all, 2, profile=True)
         del ws_all
-        core_h = sum(ms for k, ms in recs if k in ("linear_state", "linear_readout", "anchor")) / args.steps
+        core_h = sum(ms for k, ms in recs
+                     if k in ("linear_state", "linear_reduce", "linear_readout", "anchor")) / args.steps
         core_a = sum(ms for k, ms in recs_all if k == "anchor") / 2
         speedup = {"all_softmax_ms_per_step": ms_all / 2,
                    "stack": (ms_all / 2) / (ms_total / args.steps),

@@ -200,7 +200,8 @@ typedef enum {
   SVA_KERNEL_ANCHOR = 4,
   SVA_KERNEL_ROUTE = 5,
   SVA_KERNEL_KEYS = 6,
-  SVA_KERNEL_OTHER = 7
+  SVA_KERNEL_OTHER = 7,
+  SVA_KERNEL_LINEAR_REDUCE = 8
 } sva_kernel_class_t;
 
 typedef struct {

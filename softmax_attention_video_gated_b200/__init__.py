@@ -23,7 +23,7 @@ SVA_F32, SVA_BF16 = 0, 1
 SVA_STATUS_BYTES = 256
 SVA_FLAG_QK_FEATURES = 1
 KERNEL_CLASSES = ("proj_qkvg", "proj_out", "linear_state", "linear_readout", "anchor", "route",
-                  "keys", "other")
+                  "keys", "other", "linear_reduce")
 
 _c_void_p_p = ctypes.POINTER(ctypes.c_void_p)
 

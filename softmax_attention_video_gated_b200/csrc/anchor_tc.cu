@@ -5,18 +5,25 @@
 // It Works"]: Y_t = sum_s softmax_s(scale Q_t . K_s) V_s * sigmoid(G_t),
 // non-causal. FlashAttention-style: no N x N matrix is ever stored.
 //
-// One CTA per (128-query tile, head, batch); 6 warps:
-//   warp 0      TMA: the Q tile once, then 128-key K and V tiles (2 stages)
-//   warp 1      TMEM (512 columns: S0 | S1 | O); lane 0 issues the MMAs:
-//               S_j = Q K_j^T (SS, M=128 N=128) into S[j%2] and
-//               O += P_j V_j with P_j read from TMEM (TS, V MN-major)
-//   warps 2..5  softmax: thread r owns query row r (its TMEM lane); loads S_j,
-//               online max in the log2 domain, exp2, row sum, writes P_j as
-//               bf16 over the first 64 columns of S[j%2]; rescales the O row
-//               only when the running max grows by more than 2^8 (the stale
-//               max keeps every p <= 2^8, exact after the final 1/l); then the
-//               epilogue O / l * sigmoid(G) (+ residual) -> bf16.
-// The MMA of S_{j+1} and of P_{j-1} V_{j-1} overlap the softmax of S_j.
+// One CTA per pair of 128-query tiles of one (head, batch); 12 warps in three
+// warpgroups:
+//   WG0  warp 0: TMA (both Q tiles once, then 128-key K and V tiles, 2 stages);
+//        warp 1: allocates all 512 TMEM columns (tile t: S_t at 256t, O_t at
+//        256t+128) and issues every MMA from one thread. Registers shrink to 56.
+//   WG1, WG2  softmax of tile 0 and tile 1: thread r owns query row r (its
+//        TMEM lane). Registers grow to 224 so a row of S stays in registers.
+// The MMA thread ping-pongs the tiles: O_0 += P_0 V_j, S_0 = Q_0 K_{j+1}, then
+// O_1 += P_1 V_j, S_1 = Q_1 K_{j+1}, so the tensor core works on one tile while
+// the other tile's softmax runs. P (bf16) is written over the first 64 columns
+// of S and consumed straight from TMEM (A operand in TMEM); in-order execution
+// of the MMAs keeps S_{j+1} from overwriting P_j before P_j V_j has read it,
+// and the commit that reports S_{j+1} also covers P_j V_j, so a softmax warp
+// that sees S_{j+1} may rescale O.
+// Softmax per row: running max in the log2 domain, rescaled only when it grows
+// by more than 8 (p <= 2^8 otherwise, exact after the final 1/l); one FFMA per
+// element folds the scale; three of every four exponentials go to the MUFU
+// unit and one to the FMA pipe (Cody-Waite reduction and a minimax cubic, see
+// fit_exp2_poly.py), which takes load off the MUFU unit.
 #include <algorithm>
 #include <math.h>
 
@@ -30,13 +37,19 @@ constexpr int HD = 128;
 constexpr int BQ = 128, BKV = 128;
 constexpr int BOX = 128 * 128;              // [64 cols x 128 rows] bf16 = 16 KB
 constexpr int KV_STAGES = 2;
-constexpr int Q_OFF = 0;                     // 32 KB
-constexpr int KV_OFF = 2 * BOX;              // stage s: K at +s*64K, V at +s*64K+32K
+constexpr int Q_OFF = 0;                     // tile t: 32 KB at Q_OFF + t * 2 * BOX
+constexpr int KV_OFF = 4 * BOX;              // stage s: K at +s*64K, V at +s*64K+32K
 constexpr int KV_STAGE_BYTES = 4 * BOX;
 constexpr int TAIL_OFF = KV_OFF + KV_STAGES * KV_STAGE_BYTES;
+constexpr int NUM_THREADS = 384;
 constexpr int TMEM_COLS = 512;
-constexpr int S_COL0 = 0, O_COL = 256;
 constexpr float kRescaleThreshold = 8.0f;    // log2 units
+// register split: 128 threads at 56 + 256 threads at 224 = 384 threads at 168
+constexpr int kRegsProducer = 56, kRegsSoftmax = 224;
+
+// minimax cubic for 2^f on [-1/2, 1/2] with c0 = 1 (fit_exp2_poly.py);
+// max relative error 4.4e-4, five times below bf16's rounding of P
+constexpr float kP1 = 0.695766806602478f, kP2 = 0.24203051626682281f, kP3 = 0.041698750108480453f;
 
 struct AnchorTail {
   uint64_t q_full;
@@ -57,13 +70,25 @@ __device__ __forceinline__ bool drain_wait(uint64_t* bar, uint32_t parity) {
   return mbar_wait(bar, parity, &never, nullptr, 0);
 }
 
-__device__ __forceinline__ float ex2(float x) {
+__device__ __forceinline__ float ex2_mufu(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
 }
 
-__global__ void __launch_bounds__(192, 1)
+// 2^x on the FMA pipe: x = n + f with n = rint(x) (1.5 * 2^23 added and taken
+// away), 2^f by the cubic, 2^n by adding n to the exponent bits. x is clamped at
+// -127, where the result is exactly 0 (n = -127, f = 0).
+__device__ __forceinline__ float ex2_poly(float x) {
+  x = fmaxf(x, -127.0f);
+  const float t = x + 12582912.0f;
+  const float f = x - (t - 12582912.0f);
+  const float p = fmaf(fmaf(fmaf(kP3, f, kP2), f, kP1), f, 1.0f);
+  // the low bits of t hold n; the bits of 1.5 * 2^23 shifted by 23 vanish mod 2^32
+  return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
+}
+
+__global__ void __launch_bounds__(NUM_THREADS, 1)
     anchor_tc_kernel(const __grid_constant__ CUtensorMap map_q,
                      const __grid_constant__ CUtensorMap map_k,
                      const __grid_constant__ CUtensorMap map_v, int N, float scale_log2,
@@ -73,9 +98,11 @@ __global__ void __launch_bounds__(192, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
   AnchorTail* tl = reinterpret_cast<AnchorTail*>(smem + TAIL_OFF);
-  const int qt = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+  const int q0 = blockIdx.x * 2 * BQ, h = blockIdx.y, b = blockIdx.z;
   const int warp = warp_id(), lane = lane_id();
+  const int wg = warp >> 2;
   const int nkv = (N + BKV - 1) / BKV;
+  const bool has1 = q0 + BQ < N;  // the second tile holds at least one query
 
   if (threadIdx.x == 0) {
     mbar_init(&tl->q_full, 1);
@@ -108,12 +135,17 @@ __global__ void __launch_bounds__(192, 1)
   const uint32_t tmem = tl->tmem_base;
   volatile int* abort_flag = &tl->abort_flag;
 
-  if (warp == 0) {
-    if (lane == 0) {
+  if (wg == 0) {
+    warpgroup_reg_dec<kRegsProducer>();
+    if (warp == 0 && lane == 0) {
       // ------------------------------------------------ TMA producer
-      mbar_arrive_expect_tx(&tl->q_full, 2 * BOX);
-      tma_load_3d(&map_q, &tl->q_full, smem + Q_OFF, h * HD, qt * BQ, b);
-      tma_load_3d(&map_q, &tl->q_full, smem + Q_OFF + BOX, h * HD + 64, qt * BQ, b);
+      mbar_arrive_expect_tx(&tl->q_full, (has1 ? 4 : 2) * BOX);
+      tma_load_3d(&map_q, &tl->q_full, smem + Q_OFF, h * HD, q0, b);
+      tma_load_3d(&map_q, &tl->q_full, smem + Q_OFF + BOX, h * HD + 64, q0, b);
+      if (has1) {
+        tma_load_3d(&map_q, &tl->q_full, smem + Q_OFF + 2 * BOX, h * HD, q0 + BQ, b);
+        tma_load_3d(&map_q, &tl->q_full, smem + Q_OFF + 3 * BOX, h * HD + 64, q0 + BQ, b);
+      }
       int issued = 0;
       bool ok = true;
       for (int j = 0; j < nkv; ++j) {
@@ -138,21 +170,16 @@ __global__ void __launch_bounds__(192, 1)
           (void)drain_wait(&tl->k_full[i % KV_STAGES], (i / KV_STAGES) & 1);
           (void)drain_wait(&tl->v_full[i % KV_STAGES], (i / KV_STAGES) & 1);
         }
-    }
-  } else if (warp == 1) {
-    if (lane == 0) {
+    } else if (warp == 1 && lane == 0) {
       // ------------------------------------------------ MMA issuer
       constexpr uint32_t idesc_s = idesc_bf16_f32(BQ, BKV, false, false);  // Q, K: K-major
       constexpr uint32_t idesc_o = idesc_bf16_f32(BQ, HD, false, true);    // P (TMEM), V: MN-major
-      const uint32_t qaddr = smem_u32(smem + Q_OFF);
+      const int ntiles = has1 ? 2 : 1;
       bool ok = mbar_wait(&tl->q_full, 0, abort_flag, status, WHERE_ANCHOR);
-      auto issue_s = [&](int j) -> bool {
-        const int st = j % KV_STAGES;
-        if (!mbar_wait(&tl->k_full[st], (j / KV_STAGES) & 1, abort_flag, status, WHERE_ANCHOR))
-          return false;
-        tc_fence_after();
-        const uint32_t kaddr = smem_u32(smem + KV_OFF + st * KV_STAGE_BYTES);
-        const uint32_t d_tmem = tmem + S_COL0 + (j & 1) * BKV;
+      auto issue_s = [&](int t, int j) {
+        const uint32_t qaddr = smem_u32(smem + Q_OFF + t * 2 * BOX);
+        const uint32_t kaddr = smem_u32(smem + KV_OFF + (j % KV_STAGES) * KV_STAGE_BYTES);
+        const uint32_t d_tmem = tmem + t * 256;
 #pragma unroll
         for (int kk = 0; kk < HD / 16; ++kk) {
           const int bx = kk >> 2, w = kk & 3;
@@ -160,157 +187,178 @@ __global__ void __launch_bounds__(192, 1)
           const uint64_t bd = smem_desc(kaddr + bx * BOX + w * 32, 16, 1024);
           umma_ss(d_tmem, ad, bd, idesc_s, kk != 0 ? 1u : 0u);
         }
-        umma_commit(&tl->s_full[j & 1]);
-        return true;
+        umma_commit(&tl->s_full[t]);
       };
-      if (ok && nkv > 0) ok = issue_s(0);
-      for (int j = 0; j < nkv && ok; ++j) {
-        if (j + 1 < nkv && !issue_s(j + 1)) {
-          ok = false;
-          break;
-        }
-        const int st = j % KV_STAGES;
-        if (!mbar_wait(&tl->p_full[j & 1], (j >> 1) & 1, abort_flag, status, WHERE_ANCHOR) ||
-            !mbar_wait(&tl->v_full[st], (j / KV_STAGES) & 1, abort_flag, status, WHERE_ANCHOR)) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-        const uint32_t vaddr = smem_u32(smem + KV_OFF + st * KV_STAGE_BYTES + 2 * BOX);
-        const uint32_t p_tmem = tmem + S_COL0 + (j & 1) * BKV;
+      auto issue_pv = [&](int t, int j) {
+        const uint32_t vaddr =
+            smem_u32(smem + KV_OFF + (j % KV_STAGES) * KV_STAGE_BYTES + 2 * BOX);
+        const uint32_t p_tmem = tmem + t * 256;
 #pragma unroll
         for (int kk = 0; kk < BKV / 16; ++kk) {
           const uint64_t bd = smem_desc(vaddr + kk * 2048, BOX, 1024);
-          umma_ts(tmem + O_COL, p_tmem + kk * 8, bd, idesc_o, (j | kk) != 0 ? 1u : 0u);
+          umma_ts(tmem + t * 256 + 128, p_tmem + kk * 8, bd, idesc_o, (j | kk) != 0 ? 1u : 0u);
         }
-        umma_commit(&tl->o_done);
-        umma_commit(&tl->kv_empty[st]);
+      };
+      if (ok && nkv > 0) {
+        ok = mbar_wait(&tl->k_full[0], 0, abort_flag, status, WHERE_ANCHOR);
+        if (ok) {
+          tc_fence_after();
+          for (int t = 0; t < ntiles; ++t) issue_s(t, 0);
+        }
       }
+      for (int j = 0; j < nkv && ok; ++j) {
+        const int st = j % KV_STAGES;
+        const bool more = j + 1 < nkv;
+        if (!mbar_wait(&tl->v_full[st], (j / KV_STAGES) & 1, abort_flag, status, WHERE_ANCHOR) ||
+            (more && !mbar_wait(&tl->k_full[(j + 1) % KV_STAGES], ((j + 1) / KV_STAGES) & 1,
+                                abort_flag, status, WHERE_ANCHOR))) {
+          ok = false;
+          break;
+        }
+        for (int t = 0; t < ntiles; ++t) {
+          if (!mbar_wait(&tl->p_full[t], j & 1, abort_flag, status, WHERE_ANCHOR)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          issue_pv(t, j);
+          if (t == ntiles - 1) umma_commit(&tl->kv_empty[st]);
+          if (more) issue_s(t, j + 1);
+        }
+      }
+      if (ok) umma_commit(&tl->o_done);
       umma_commit(&tl->drain);
       (void)drain_wait(&tl->drain, 0);
     }
   } else {
-    // ------------------------------------------------ softmax + epilogue (warps 2..5)
+    warpgroup_reg_inc<kRegsSoftmax>();
+    // ------------------------------------------------ softmax + epilogue (WG1: tile 0, WG2: tile 1)
+    const int t = wg - 1;
     const int q = warp & 3;
     const int r = q * 32 + lane;
     const uint32_t lane_base = static_cast<uint32_t>(q * 32) << 16;
-    float m = -INFINITY;  // running (possibly stale) max of scaled logits, log2 units
-    float l = 0.f;
-    bool ok = true;
-    for (int j = 0; j < nkv; ++j) {
-      bool w = mbar_wait(&tl->s_full[j & 1], (j >> 1) & 1, abort_flag, status, WHERE_ANCHOR);
-      if (!__all_sync(0xffffffffu, w)) {
-        ok = false;
-        break;
-      }
-      tc_fence_after();
-      const uint32_t sc = tmem + lane_base + S_COL0 + (j & 1) * BKV;
-      float s[BKV];
-#pragma unroll
-      for (int c = 0; c < BKV; c += 32) {
-        uint32_t v[32];
-        tmem_ld32(sc + c, v);
-        tmem_wait_ld();
-#pragma unroll
-        for (int i = 0; i < 32; ++i) s[c + i] = __uint_as_float(v[i]) * scale_log2;
-      }
-      const int valid = N - j * BKV;  // keys of this block inside the sequence
-      if (valid < BKV) {
-#pragma unroll
-        for (int i = 0; i < BKV; ++i)
-          if (i >= valid) s[i] = -INFINITY;
-      }
-      float mx = s[0];
-#pragma unroll
-      for (int i = 1; i < BKV; ++i) mx = fmaxf(mx, s[i]);
-      float m_use = m;
-      float factor = 1.f;
-      const bool grow = mx > m + kRescaleThreshold;
-      if (grow) {
-        factor = (m == -INFINITY) ? 0.f : ex2(m - mx);
-        m_use = mx;
-      }
-      // rescale the O row (only rows whose max grew; warps where none did skip it)
-      if (j > 0 && __any_sync(0xffffffffu, grow)) {
-        bool wo = mbar_wait(&tl->o_done, (j - 1) & 1, abort_flag, status, WHERE_ANCHOR);
-        if (!__all_sync(0xffffffffu, wo)) {
+    const uint32_t s_col = tmem + lane_base + t * 256;
+    const uint32_t o_col = s_col + 128;
+    if (t == 0 || has1) {
+      float m = -INFINITY;  // running (possibly stale) max of scaled logits, log2 units
+      float l = 0.f;
+      bool ok = true;
+      for (int j = 0; j < nkv; ++j) {
+        bool w = mbar_wait(&tl->s_full[t], j & 1, abort_flag, status, WHERE_ANCHOR);
+        if (!__all_sync(0xffffffffu, w)) {
           ok = false;
           break;
         }
         tc_fence_after();
-#pragma unroll 1
-        for (int c = 0; c < HD; c += 32) {
-          uint32_t v[32];
-          tmem_ld32(tmem + lane_base + O_COL + c, v);
-          tmem_wait_ld();
+        uint32_t v[4][32];
+        tmem_ld32(s_col, v[0]);
+        tmem_ld32(s_col + 32, v[1]);
+        tmem_ld32(s_col + 64, v[2]);
+        tmem_ld32(s_col + 96, v[3]);
+        tmem_wait_ld();
+        float s[BKV];
 #pragma unroll
-          for (int i = 0; i < 32; ++i) v[i] = __float_as_uint(__uint_as_float(v[i]) * factor);
-          tmem_st32(tmem + lane_base + O_COL + c, v);
+        for (int i = 0; i < BKV; ++i) s[i] = __uint_as_float(v[i >> 5][i & 31]);
+        const int valid = N - j * BKV;  // keys of this block inside the sequence
+        if (valid < BKV) {
+#pragma unroll
+          for (int i = 0; i < BKV; ++i)
+            if (i >= valid) s[i] = -INFINITY;
+        }
+        float mx8[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) mx8[i] = s[i];
+#pragma unroll
+        for (int i = 8; i < BKV; ++i) mx8[i & 7] = fmaxf(mx8[i & 7], s[i]);
+        const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+                               fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7]))) *
+                         scale_log2;
+        const bool grow = mx > m + kRescaleThreshold;
+        float factor = 1.f;
+        if (grow) {
+          factor = (m == -INFINITY) ? 0.f : ex2_mufu(m - mx);
+          m = mx;
+        }
+        // O of this tile is complete up to block j-1 here: the commit that
+        // reported S_j also covers P_{j-1} V_{j-1}
+        if (j > 0 && __any_sync(0xffffffffu, grow)) {
+#pragma unroll 1
+          for (int c = 0; c < HD; c += 32) {
+            uint32_t o[32];
+            tmem_ld32(o_col + c, o);
+            tmem_wait_ld();
+#pragma unroll
+            for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * factor);
+            tmem_st32(o_col + c, o);
+          }
+        }
+        l *= factor;
+        const float neg_m = -m;
+        float acc[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) acc[i] = 0.f;
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          uint32_t pk[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            const float x0 = fmaf(s[32 * c + 2 * i], scale_log2, neg_m);
+            const float x1 = fmaf(s[32 * c + 2 * i + 1], scale_log2, neg_m);
+            const float p0 = ex2_mufu(x0);
+            const float p1 = (i & 1) ? ex2_poly(x1) : ex2_mufu(x1);  // 1 in 4 on the FMA pipe
+            acc[i & 7] += p0 + p1;
+            pk[i] = pack_bf16x2(p0, p1);
+          }
+          tmem_st16(s_col + 16 * c, pk);
         }
         tmem_wait_st();
+        l += ((acc[0] + acc[1]) + (acc[2] + acc[3])) + ((acc[4] + acc[5]) + (acc[6] + acc[7]));
+        tc_fence_before();
+        mbar_arrive(&tl->p_full[t]);
       }
-      l *= factor;
-      m = m_use;
-      float rs = 0.f;
-#pragma unroll
-      for (int c = 0; c < BKV; c += 32) {
-        uint32_t pk[16];
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          const float p0 = ex2(s[c + 2 * i] - m);
-          const float p1 = ex2(s[c + 2 * i + 1] - m);
-          rs += p0 + p1;
-          pk[i] = pack_bf16x2(p0, p1);
-        }
-        tmem_st16(sc + c / 2, pk);
+      if (ok && nkv > 0) {
+        bool w = mbar_wait(&tl->o_done, 0, abort_flag, status, WHERE_ANCHOR);
+        ok = __all_sync(0xffffffffu, w);
       }
-      tmem_wait_st();
-      l += rs;
-      tc_fence_before();
-      mbar_arrive(&tl->p_full[j & 1]);
-    }
-    if (ok && nkv > 0) {
-      bool w = mbar_wait(&tl->o_done, (nkv - 1) & 1, abort_flag, status, WHERE_ANCHOR);
-      ok = __all_sync(0xffffffffu, w);
-    }
-    if (ok) {
-      tc_fence_after();
-      const int t = qt * BQ + r;
-      const float inv = 1.0f / l;
-      const bool row_ok = t < N;
-      const int64_t row = static_cast<int64_t>(b) * N + t;
+      if (ok) {
+        tc_fence_after();
+        const int row_t = q0 + t * BQ + r;
+        const float inv = 1.0f / l;
+        const bool row_ok = row_t < N;
+        const int64_t row = static_cast<int64_t>(b) * N + row_t;
 #pragma unroll 1
-      for (int c = 0; c < HD; c += 32) {
-        uint32_t v[32];
-        tmem_ld32(tmem + lane_base + O_COL + c, v);
-        tmem_wait_ld();
-        if (!row_ok) continue;
-        const __nv_bfloat16* gp = gate + row * ldg + h * HD + c;
-        __nv_bfloat16* op = out + row * ldo + h * HD + c;
+        for (int c = 0; c < HD; c += 32) {
+          uint32_t o[32];
+          tmem_ld32(o_col + c, o);
+          tmem_wait_ld();
+          if (!row_ok) continue;
+          const __nv_bfloat16* gp = gate + row * ldg + h * HD + c;
+          __nv_bfloat16* op = out + row * ldo + h * HD + c;
 #pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          const uint4 gv = *reinterpret_cast<const uint4*>(gp + 8 * k);
-          const float gg[8] = {bf16lo_to_f32(gv.x), bf16hi_to_f32(gv.x), bf16lo_to_f32(gv.y),
-                               bf16hi_to_f32(gv.y), bf16lo_to_f32(gv.z), bf16hi_to_f32(gv.z),
-                               bf16lo_to_f32(gv.w), bf16hi_to_f32(gv.w)};
-          float y[8];
+          for (int k = 0; k < 4; ++k) {
+            const uint4 gv = *reinterpret_cast<const uint4*>(gp + 8 * k);
+            const float gg[8] = {bf16lo_to_f32(gv.x), bf16hi_to_f32(gv.x), bf16lo_to_f32(gv.y),
+                                 bf16hi_to_f32(gv.y), bf16lo_to_f32(gv.z), bf16hi_to_f32(gv.z),
+                                 bf16lo_to_f32(gv.w), bf16hi_to_f32(gv.w)};
+            float y[8];
 #pragma unroll
-          for (int e = 0; e < 8; ++e)
-            y[e] = __uint_as_float(v[8 * k + e]) * inv * fast_sigmoid(gg[e]);
-          if (residual != nullptr) {
-            const uint4 rv =
-                *reinterpret_cast<const uint4*>(residual + row * ldr + h * HD + c + 8 * k);
-            y[0] += bf16lo_to_f32(rv.x); y[1] += bf16hi_to_f32(rv.x);
-            y[2] += bf16lo_to_f32(rv.y); y[3] += bf16hi_to_f32(rv.y);
-            y[4] += bf16lo_to_f32(rv.z); y[5] += bf16hi_to_f32(rv.z);
-            y[6] += bf16lo_to_f32(rv.w); y[7] += bf16hi_to_f32(rv.w);
+            for (int e = 0; e < 8; ++e)
+              y[e] = __uint_as_float(o[8 * k + e]) * inv * fast_sigmoid(gg[e]);
+            if (residual != nullptr) {
+              const uint4 rv =
+                  *reinterpret_cast<const uint4*>(residual + row * ldr + h * HD + c + 8 * k);
+              y[0] += bf16lo_to_f32(rv.x); y[1] += bf16hi_to_f32(rv.x);
+              y[2] += bf16lo_to_f32(rv.y); y[3] += bf16hi_to_f32(rv.y);
+              y[4] += bf16lo_to_f32(rv.z); y[5] += bf16hi_to_f32(rv.z);
+              y[6] += bf16lo_to_f32(rv.w); y[7] += bf16hi_to_f32(rv.w);
+            }
+            uint4 ov;
+            ov.x = pack_bf16x2(y[0], y[1]);
+            ov.y = pack_bf16x2(y[2], y[3]);
+            ov.z = pack_bf16x2(y[4], y[5]);
+            ov.w = pack_bf16x2(y[6], y[7]);
+            *reinterpret_cast<uint4*>(op + 8 * k) = ov;
           }
-          uint4 o;
-          o.x = pack_bf16x2(y[0], y[1]);
-          o.y = pack_bf16x2(y[2], y[3]);
-          o.z = pack_bf16x2(y[4], y[5]);
-          o.w = pack_bf16x2(y[6], y[7]);
-          *reinterpret_cast<uint4*>(op + 8 * k) = o;
         }
       }
     }
@@ -347,8 +395,8 @@ cudaError_t anchor_bf16(const sva_attn_args& a, int* status, cudaStream_t s) {
   cudaError_t e = cudaFuncSetAttribute(anchor_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(kAnchorSmem));
   if (e != cudaSuccess) return e;
-  dim3 grid((a.N + BQ - 1) / BQ, a.H, a.B);
-  anchor_tc_kernel<<<grid, 192, kAnchorSmem, s>>>(
+  dim3 grid((a.N + 2 * BQ - 1) / (2 * BQ), a.H, a.B);
+  anchor_tc_kernel<<<grid, NUM_THREADS, kAnchorSmem, s>>>(
       mq, mk, mv, a.N, scale_log2, static_cast<const __nv_bfloat16*>(a.gate), a.ldg,
       static_cast<const __nv_bfloat16*>(a.residual), a.ldr, static_cast<__nv_bfloat16*>(a.out),
       a.ldo, status);

@@ -288,7 +288,7 @@ cudaError_t linear_f32(const sva_attn_args& a, int* status, void* scratch, cudaS
     if (e != cudaSuccess) return e;
   }
   {
-    ProfScope ps(prof, s, SVA_KERNEL_LINEAR_STATE);
+    ProfScope ps(prof, s, SVA_KERNEL_LINEAR_REDUCE);
     lin_reduce_f32_kernel<<<a.B * a.H, 256, 0, s>>>(partial, state, p.n_chunks, elems);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;

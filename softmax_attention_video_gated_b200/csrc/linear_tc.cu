@@ -248,28 +248,42 @@ __global__ void __launch_bounds__(192, 1)
 // ------------------------------------------------------------------ reduce
 // state_op[bh] = bf16 [144][128]: rows 0..127 = S^T (row n = d_v, column k =
 // d_k), row 128 = bf16(z), row 129 = bf16(z - bf16(z)), rows 130..143 = 0.
+// One CTA per 32x32 tile of S (16 per head): sums the chunk partials in chunk
+// order (deterministic) and writes the tile transposed through shared memory.
 __global__ void __launch_bounds__(256) lin_reduce_bf16_kernel(const float* __restrict__ partial,
                                                               __nv_bfloat16* __restrict__ state_op,
                                                               int n_chunks) {
-  const int64_t bh = blockIdx.x;
+  __shared__ float tile[32][33];
+  const int64_t bh = blockIdx.y;
+  const int ki = blockIdx.x >> 2, ni = blockIdx.x & 3;
+  const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;
   const int elems = HD * HD + HD;
   const float* p = partial + bh * n_chunks * elems;
   __nv_bfloat16* o = state_op + bh * STATE_ROWS * HD;
-  for (int e = threadIdx.x; e < HD * HD; e += 256) {
-    float s = 0.f;
-    for (int c = 0; c < n_chunks; ++c) s += p[static_cast<int64_t>(c) * elems + e];
-    const int k = e / HD, n = e % HD;
-    o[n * HD + k] = __float2bfloat16_rn(s);
+#pragma unroll
+  for (int r = 0; r < 4; ++r) {
+    const int k = ki * 32 + ty + 8 * r, n = ni * 32 + tx;
+    float acc = 0.f;
+    for (int c = 0; c < n_chunks; ++c) acc += p[static_cast<int64_t>(c) * elems + k * HD + n];
+    tile[ty + 8 * r][tx] = acc;
   }
-  for (int e = threadIdx.x; e < HD; e += 256) {
-    float s = 0.f;
-    for (int c = 0; c < n_chunks; ++c) s += p[static_cast<int64_t>(c) * elems + HD * HD + e];
-    const __nv_bfloat16 hi = __float2bfloat16_rn(s);
-    o[HD * HD + e] = hi;
-    o[(HD + 1) * HD + e] = __float2bfloat16_rn(s - __bfloat162float(hi));
+  __syncthreads();
+#pragma unroll
+  for (int r = 0; r < 4; ++r) {
+    const int n = ni * 32 + ty + 8 * r, k = ki * 32 + tx;
+    o[n * HD + k] = __float2bfloat16_rn(tile[tx][ty + 8 * r]);
   }
-  for (int e = threadIdx.x; e < (STATE_ROWS - HD - 2) * HD; e += 256)
-    o[(HD + 2) * HD + e] = __float2bfloat16_rn(0.f);
+  if (blockIdx.x == 0) {
+    for (int e = threadIdx.x; e < HD; e += 256) {
+      float acc = 0.f;
+      for (int c = 0; c < n_chunks; ++c) acc += p[static_cast<int64_t>(c) * elems + HD * HD + e];
+      const __nv_bfloat16 hi = __float2bfloat16_rn(acc);
+      o[HD * HD + e] = hi;
+      o[(HD + 1) * HD + e] = __float2bfloat16_rn(acc - __bfloat162float(hi));
+    }
+    for (int e = threadIdx.x; e < (STATE_ROWS - HD - 2) * HD; e += 256)
+      o[(HD + 2) * HD + e] = __float2bfloat16_rn(0.f);
+  }
 }
 
 // ------------------------------------------------------------------ read-out
@@ -526,8 +540,8 @@ cudaError_t linear_bf16(const sva_attn_args& a, int* status, void* scratch, cuda
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
   {
-    ProfScope ps(prof, s, SVA_KERNEL_LINEAR_STATE);
-    lin_reduce_bf16_kernel<<<a.B * a.H, 256, 0, s>>>(partial, state, p.n_chunks);
+    ProfScope ps(prof, s, SVA_KERNEL_LINEAR_REDUCE);
+    lin_reduce_bf16_kernel<<<dim3(16, a.B * a.H), 256, 0, s>>>(partial, state, p.n_chunks);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
   ProfScope ps(prof, s, SVA_KERNEL_LINEAR_READOUT);

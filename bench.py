@@ -364,13 +364,22 @@ def run_case(args):
             ws = sva.workspace(sva.sva_linear_attn_workspace_bytes(B, N, H, d, sva.SVA_BF16))
             fn = lambda: sva.sva_linear_attn_fwd(q, k, v, g, out, H, ws=ws)  # noqa: E731
             work, unit = 10.0 * B * N * D, "GB/s"
-    else:
+    elif args.case == "gemm":
         M, K, Nout = B * N, D, 4 * D
         x = W.normal_torch((M, K), 1.0, seed, W.TAG_X, "bf16")
         w = W.normal_torch((Nout, K), 1.0 / math.sqrt(K), seed, W.TAG_WQKVG, "bf16")
         y = torch.empty(M, Nout, device="cuda", dtype=torch.bfloat16)
         ws = sva.workspace(256)
         fn = lambda: sva.sva_projection_fwd(x, w, y, ws=ws)  # noqa: E731
+        work, unit = 2.0 * M * K * Nout, "TFLOP/s"
+    else:  # proj_out: h += x W_o^T with the bf16 copy of h, as in the stack
+        M, K, Nout = B * N, D, D
+        x = W.normal_torch((M, K), 1.0, seed, W.TAG_X, "bf16")
+        w = W.normal_torch((Nout, K), 1.0 / math.sqrt(K), seed, W.TAG_WO, "bf16")
+        hs = W.normal_torch((M, Nout), 1.0, seed, W.TAG_V, "f32")
+        hc = torch.empty(M, Nout, device="cuda", dtype=torch.bfloat16)
+        ws = sva.workspace(256)
+        fn = lambda: sva.sva_projection_residual_fwd(x, w, hs, hc, ws=ws)  # noqa: E731
         work, unit = 2.0 * M * K * Nout, "TFLOP/s"
     for _ in range(args.warmup):
         fn()
@@ -400,7 +409,7 @@ def main():
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-all-softmax", action="store_true")
-    ap.add_argument("--case", choices=("anchor", "linear", "gemm"),
+    ap.add_argument("--case", choices=("anchor", "linear", "gemm", "proj_out"),
                     help="time one kernel class alone instead of the stack")
     ap.add_argument("--B", type=int, default=1)
     ap.add_argument("--N", type=int, default=19320)

@@ -2,16 +2,25 @@
 // cores: C = A B^T with A [M, K] (activations) and B [N, K] (weights in the
 // [out, in] layout of a linear layer), both K-major, fp32 accumulation in TMEM.
 //
-// Persistent kernel, one CTA per SM, warp-specialised:
-//   warp 0      TMA producer: 128x64 A and 256x64 B tiles (128-byte swizzle)
-//               into a 4-stage shared-memory ring;
-//   warp 1      allocates 512 TMEM columns; lane 0 issues tcgen05.mma
-//               (M=128, N=256, K=16) into one of two 256-column accumulators;
-//   warps 2..5  epilogue: tcgen05.ld of their 32-lane quadrant, then either a
-//               bf16 store (optional ReLU on the leading columns, the feature
-//               map phi of the linear layers) or the residual update
-//               h += C (fp32) with an optional bf16 copy of h.
-// Two accumulators let the epilogue of tile i overlap the main loop of i+1.
+// Persistent kernel on clusters of two CTAs (one CTA per SM). A cluster owns
+// 256 x 256 output tiles; the pair shares each tcgen05.mma (cta_group::2):
+// CTA r loads rows [128r, 128r+128) of the A tile and rows [128r, 128r+128) of
+// the B tile (its half of N), so a k-block costs each CTA 32 KB of shared
+// memory instead of the 48 KB a single-CTA 128 x 256 tile needs. Per CTA:
+//   warp 0      TMA producer: 128x64 A and 128x64 B boxes (128-byte swizzle)
+//               into a 6-stage ring; completion is counted on the rank-0 CTA's
+//               barrier, which expects both CTAs' bytes;
+//   warp 1      allocates 512 TMEM columns (pair allocation); on rank 0 one
+//               lane issues M=256 N=256 K=16 MMAs into one of two 256-column
+//               accumulators and multicasts its commits to both CTAs;
+//   warps 2..5  epilogue of this CTA's 128 rows: tcgen05.ld, then a transpose
+//               through shared memory so global reads and writes are
+//               row-contiguous; either a bf16 store (ReLU on leading columns,
+//               the feature map phi of the linear layers) or the residual
+//               update h += C (fp32) with an optional bf16 copy of h. Each warp
+//               releases the accumulator on rank 0's barrier.
+// Tiles run in groups of whole M-tile columns so one wave touches few A rows
+// and few B rows and both stay in L2.
 #include <algorithm>
 
 #include "common.cuh"
@@ -20,42 +29,76 @@
 namespace sva {
 namespace {
 
-constexpr int BM = 128, BN = 256, BK = 64, STAGES = 4;
-constexpr int A_STAGE = BM * BK * 2;              // 16 KB
-constexpr int B_STAGE = BN * BK * 2;              // 32 KB
-constexpr int STAGE_BYTES = A_STAGE + B_STAGE;    // 48 KB
-constexpr int TMEM_COLS = 2 * BN;                 // two fp32 accumulators
+constexpr int BM = 256, BN = 256, BK = 64, MAX_STAGES = 6;
+constexpr int HALF = 128;                          // rows of A (and of B) per CTA
+constexpr int A_STAGE = HALF * BK * 2;             // 16 KB
+constexpr int B_STAGE = HALF * BK * 2;             // 16 KB
+constexpr int STAGE_BYTES = A_STAGE + B_STAGE;     // 32 KB per CTA
+constexpr int TMEM_COLS = 2 * BN;                  // two fp32 accumulators
 constexpr int NUM_THREADS = 192;
+// EPI_STORE epilogue: a 32 x 32 fp32 transpose buffer per warp
+constexpr int STG_STRIDE = 36;                     // fp32 words per staged row (16-byte aligned)
+constexpr int STG_WARP_BYTES = 32 * STG_STRIDE * 4;
+// EPI_RESIDUAL epilogue: per warp two slots of a 32 x 32 fp32 tile of h
+// (128-byte swizzle) and two of its 32 x 32 bf16 copy (64-byte swizzle)
+constexpr int RES_H_BYTES = 32 * 32 * 4, RES_C_BYTES = 32 * 32 * 2;
+constexpr int RES_WARP_BYTES = 2 * RES_H_BYTES + 2 * RES_C_BYTES;  // 12 KB
+
+template <int EPI>
+struct Layout {
+  static constexpr int STAGES = EPI == EPI_STORE ? 6 : 5;
+  static constexpr int EPI_OFF = STAGES * STAGE_BYTES;
+  static constexpr int TAIL_OFF = EPI_OFF + 4 * (EPI == EPI_STORE ? STG_WARP_BYTES : RES_WARP_BYTES);
+};
 
 struct GemmTail {
-  uint64_t full[STAGES];
-  uint64_t empty[STAGES];
+  uint64_t full[MAX_STAGES];
+  uint64_t empty[MAX_STAGES];
   uint64_t acc_full[2];
   uint64_t acc_empty[2];
+  uint64_t hbar[4][2];  // EPI_RESIDUAL: h chunk loads, per epilogue warp and slot
   uint64_t drain;
   uint32_t tmem_base;
   int abort_flag;
 };
 
-constexpr size_t kGemmSmem = 1024 + STAGES * STAGE_BYTES + sizeof(GemmTail);
+template <int EPI>
+constexpr size_t gemm_smem() {
+  return 1024 + Layout<EPI>::TAIL_OFF + sizeof(GemmTail);
+}
 
 __device__ __forceinline__ bool drain_wait(uint64_t* bar, uint32_t parity) {
   int never = 0;
   return mbar_wait(bar, parity, &never, nullptr, 0);
 }
 
+__device__ __forceinline__ void tile_coords(int tile, int m_tiles, int n_tiles, int group,
+                                            int& m_blk, int& n_blk) {
+  const int per_group = group * n_tiles;
+  const int g = tile / per_group, w = tile % per_group;
+  const int m0 = g * group;
+  const int gs = min(group, m_tiles - m0);
+  m_blk = m0 + w % gs;
+  n_blk = w / gs;
+}
+
 template <int EPI>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     gemm_bf16_tc_kernel(const __grid_constant__ CUtensorMap map_a,
-                        const __grid_constant__ CUtensorMap map_b, GemmArgs g) {
+                        const __grid_constant__ CUtensorMap map_b,
+                        const __grid_constant__ CUtensorMap map_h,
+                        const __grid_constant__ CUtensorMap map_c, GemmArgs g, int group) {
+  constexpr int STAGES = Layout<EPI>::STAGES;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
   uint8_t* sA = smem;
   uint8_t* sB = smem + STAGES * A_STAGE;
-  GemmTail* tl = reinterpret_cast<GemmTail*>(smem + STAGES * STAGE_BYTES);
+  GemmTail* tl = reinterpret_cast<GemmTail*>(smem + Layout<EPI>::TAIL_OFF);
 
   const int warp = warp_id(), lane = lane_id();
+  const uint32_t rank = cluster_ctarank();
+  const int cluster = blockIdx.x >> 1, n_clusters = gridDim.x >> 1;
   const int m_tiles = static_cast<int>((g.M + BM - 1) / BM);
   const int n_tiles = static_cast<int>((g.N + BN - 1) / BN);
   const int num_tiles = m_tiles * n_tiles;
@@ -68,43 +111,51 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(&tl->acc_full[a], 1);
-      mbar_init(&tl->acc_empty[a], 4);
+      mbar_init(&tl->acc_empty[a], 8);  // 4 epilogue warps in each CTA of the pair
     }
+    for (int w = 0; w < 4; ++w)
+      for (int sl = 0; sl < 2; ++sl) mbar_init(&tl->hbar[w][sl], 1);
     mbar_init(&tl->drain, 1);
     tl->abort_flag = 0;
     fence_mbar_init();
   }
   if (warp == 1) {
-    tmem_alloc(&tl->tmem_base, TMEM_COLS);
-    tmem_relinquish();
+    tmem_alloc_pair(&tl->tmem_base, TMEM_COLS);
+    tmem_relinquish_pair();
   }
   if (warp == 0 && lane == 0) {
     tma_prefetch_desc(&map_a);
     tma_prefetch_desc(&map_b);
+    if (EPI == EPI_RESIDUAL) {
+      tma_prefetch_desc(&map_h);
+      tma_prefetch_desc(&map_c);
+    }
   }
   tc_fence_before();
-  __syncthreads();
+  cluster_sync();  // both CTAs' barriers exist before either signals the other's
   tc_fence_after();
   const uint32_t tmem_base = tl->tmem_base;
   volatile int* abort_flag = &tl->abort_flag;
 
   if (warp == 0) {
     if (lane == 0) {
-      // ------------------------------------------------ TMA producer
+      // ------------------------------------------------ TMA producer (both CTAs)
       int stage = 0;
       uint32_t phase = 0;
       int64_t issued = 0;
       bool ok = true;
-      for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
-        const int m_blk = tile / n_tiles, n_blk = tile % n_tiles;
+      for (int tile = cluster; tile < num_tiles && ok; tile += n_clusters) {
+        int m_blk, n_blk;
+        tile_coords(tile, m_tiles, n_tiles, group, m_blk, n_blk);
         for (int kb = 0; kb < k_blocks; ++kb) {
           if (!mbar_wait(&tl->empty[stage], phase ^ 1, abort_flag, g.status, WHERE_GEMM)) {
             ok = false;
             break;
           }
-          mbar_arrive_expect_tx(&tl->full[stage], STAGE_BYTES);
-          tma_load_2d(&map_a, &tl->full[stage], sA + stage * A_STAGE, kb * BK, m_blk * BM);
-          tma_load_2d(&map_b, &tl->full[stage], sB + stage * B_STAGE, kb * BK, n_blk * BN);
+          const uint32_t full0 = cluster_map(&tl->full[stage], 0);
+          if (rank == 0) mbar_arrive_expect_tx(&tl->full[stage], 2 * STAGE_BYTES);
+          tma_load_2d_pair(&map_a, full0, sA + stage * A_STAGE, kb * BK, m_blk * BM + rank * HALF);
+          tma_load_2d_pair(&map_b, full0, sB + stage * B_STAGE, kb * BK, n_blk * BN + rank * HALF);
           ++issued;
           if (++stage == STAGES) {
             stage = 0;
@@ -112,21 +163,21 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           }
         }
       }
-      if (!ok) {
-        // abort: let every load still in flight land before the CTA exits
+      if (!ok && rank == 0) {
+        // abort: let the loads still in flight land before the CTA exits
         for (int64_t i = issued > STAGES ? issued - STAGES : 0; i < issued; ++i)
           (void)drain_wait(&tl->full[i % STAGES], static_cast<uint32_t>((i / STAGES) & 1));
       }
     }
   } else if (warp == 1) {
-    if (lane == 0) {
-      // ------------------------------------------------ MMA issuer
+    if (lane == 0 && rank == 0) {
+      // ------------------------------------------------ MMA issuer (rank 0 only)
       constexpr uint32_t idesc = idesc_bf16_f32(BM, BN, false, false);
       int stage = 0;
       uint32_t phase = 0;
       int local = 0;
       bool ok = true;
-      for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x, ++local) {
+      for (int tile = cluster; tile < num_tiles && ok; tile += n_clusters, ++local) {
         const int acc = local & 1;
         const uint32_t acc_phase = (local >> 1) & 1;
         if (!mbar_wait(&tl->acc_empty[acc], acc_phase ^ 1, abort_flag, g.status, WHERE_GEMM)) {
@@ -147,111 +198,213 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           for (int kk = 0; kk < BK / 16; ++kk) {
             const uint64_t ad = smem_desc(a_addr + kk * 32, 16, 1024);
             const uint64_t bd = smem_desc(b_addr + kk * 32, 16, 1024);
-            umma_ss(d_tmem, ad, bd, idesc, (kb | kk) != 0 ? 1u : 0u);
+            umma_ss_pair(d_tmem, ad, bd, idesc, (kb | kk) != 0 ? 1u : 0u);
           }
-          umma_commit(&tl->empty[stage]);
+          umma_commit_pair(&tl->empty[stage], 0x3);
           if (++stage == STAGES) {
             stage = 0;
             phase ^= 1;
           }
         }
-        if (ok) umma_commit(&tl->acc_full[acc]);
+        if (ok) umma_commit_pair(&tl->acc_full[acc], 0x3);
       }
       // every MMA issued above completes before TMEM is released
-      umma_commit(&tl->drain);
+      umma_commit_pair(&tl->drain, 0x1);
       (void)drain_wait(&tl->drain, 0);
     }
-  } else {
-    // ------------------------------------------------ epilogue (warps 2..5)
+  } else if (EPI == EPI_STORE) {
+    // ------------------------------------------------ epilogue (warps 2..5, both CTAs)
     const int q = warp & 3;  // TMEM lane quadrant of this warp
+    float* stg = reinterpret_cast<float*>(smem + Layout<EPI>::EPI_OFF + q * STG_WARP_BYTES);
+    const uint32_t acc_empty0[2] = {cluster_map(&tl->acc_empty[0], 0),
+                                    cluster_map(&tl->acc_empty[1], 0)};
     int local = 0;
-    for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++local) {
+    for (int tile = cluster; tile < num_tiles; tile += n_clusters, ++local) {
       const int acc = local & 1;
       const uint32_t acc_phase = (local >> 1) & 1;
       const bool w = mbar_wait(&tl->acc_full[acc], acc_phase, abort_flag, g.status, WHERE_GEMM);
       if (!__all_sync(0xffffffffu, w)) break;
       tc_fence_after();
-      const int m_blk = tile / n_tiles, n_blk = tile % n_tiles;
-      const int64_t row = static_cast<int64_t>(m_blk) * BM + q * 32 + lane;
-      const bool row_ok = row < g.M;
+      int m_blk, n_blk;
+      tile_coords(tile, m_tiles, n_tiles, group, m_blk, n_blk);
+      const int64_t row0 = static_cast<int64_t>(m_blk) * BM + rank * HALF + q * 32;
 #pragma unroll 1
       for (int cc = 0; cc < BN; cc += 32) {
         uint32_t r[32];
         tmem_ld32(tmem_base + (static_cast<uint32_t>(q * 32) << 16) + acc * BN + cc, r);
         tmem_wait_ld();
         const int64_t col0 = static_cast<int64_t>(n_blk) * BN + cc;
-        if (!row_ok || col0 >= g.N) continue;
-        const bool full = col0 + 32 <= g.N;
-        if (EPI == EPI_STORE) {
-          float v[32];
+        if (col0 >= g.N || row0 >= g.M) continue;  // warp-uniform
+        // stage the warp's 32 rows x 32 columns (thread = row), then read back
+        // four rows per instruction, eight threads per 128-byte row
 #pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            v[i] = __uint_as_float(r[i]);
-            if (col0 + i < g.relu_cols) v[i] = relu_f(v[i]);
-          }
-          __nv_bfloat16* out = static_cast<__nv_bfloat16*>(g.c) + row * g.ldc + col0;
-          if (full) {
-#pragma unroll
-            for (int i = 0; i < 32; i += 8) {
-              uint4 w;
-              w.x = pack_bf16x2(v[i], v[i + 1]);
-              w.y = pack_bf16x2(v[i + 2], v[i + 3]);
-              w.z = pack_bf16x2(v[i + 4], v[i + 5]);
-              w.w = pack_bf16x2(v[i + 6], v[i + 7]);
-              *reinterpret_cast<uint4*>(out + i) = w;
-            }
-          } else {
-            for (int i = 0; col0 + i < g.N; ++i) out[i] = __float2bfloat16_rn(v[i]);
-          }
-        } else {
-          float* hp = g.h + row * g.ldh + col0;
-          float v[32];
-          if (full) {
-#pragma unroll
-            for (int i = 0; i < 32; i += 4) {
-              float4 x = *reinterpret_cast<const float4*>(hp + i);
-              x.x += __uint_as_float(r[i]);
-              x.y += __uint_as_float(r[i + 1]);
-              x.z += __uint_as_float(r[i + 2]);
-              x.w += __uint_as_float(r[i + 3]);
-              *reinterpret_cast<float4*>(hp + i) = x;
-              v[i] = x.x; v[i + 1] = x.y; v[i + 2] = x.z; v[i + 3] = x.w;
-            }
-            if (g.h_copy != nullptr) {
-              __nv_bfloat16* cp = static_cast<__nv_bfloat16*>(g.h_copy) + row * g.ldhc + col0;
-#pragma unroll
-              for (int i = 0; i < 32; i += 8) {
-                uint4 w;
-                w.x = pack_bf16x2(v[i], v[i + 1]);
-                w.y = pack_bf16x2(v[i + 2], v[i + 3]);
-                w.z = pack_bf16x2(v[i + 4], v[i + 5]);
-                w.w = pack_bf16x2(v[i + 6], v[i + 7]);
-                *reinterpret_cast<uint4*>(cp + i) = w;
+        for (int k = 0; k < 8; ++k)
+          *reinterpret_cast<uint4*>(stg + lane * STG_STRIDE + 4 * k) =
+              make_uint4(r[4 * k], r[4 * k + 1], r[4 * k + 2], r[4 * k + 3]);
+        __syncwarp();
+        const int sub = lane >> 3, c4 = (lane & 7) * 4;
+        const int64_t col = col0 + c4;
+        const bool col_ok = col + 4 <= g.N;
+#pragma unroll 2
+        for (int it = 0; it < 8; ++it) {
+          const int rr = it * 4 + sub;
+          const int64_t row = row0 + rr;
+          float4 v = *reinterpret_cast<const float4*>(stg + rr * STG_STRIDE + c4);
+          if (row < g.M) {
+            {
+              if (col + 0 < g.relu_cols) v.x = relu_f(v.x);
+              if (col + 1 < g.relu_cols) v.y = relu_f(v.y);
+              if (col + 2 < g.relu_cols) v.z = relu_f(v.z);
+              if (col + 3 < g.relu_cols) v.w = relu_f(v.w);
+              __nv_bfloat16* out = static_cast<__nv_bfloat16*>(g.c) + row * g.ldc + col;
+              if (col_ok) {
+                *reinterpret_cast<uint2*>(out) =
+                    make_uint2(pack_bf16x2(v.x, v.y), pack_bf16x2(v.z, v.w));
+              } else {
+                const float vv[4] = {v.x, v.y, v.z, v.w};
+                for (int e = 0; e < 4 && col + e < g.N; ++e) out[e] = __float2bfloat16_rn(vv[e]);
               }
-            }
-          } else {
-            for (int i = 0; col0 + i < g.N; ++i) {
-              const float x = hp[i] + __uint_as_float(r[i]);
-              hp[i] = x;
-              if (g.h_copy != nullptr)
-                static_cast<__nv_bfloat16*>(g.h_copy)[row * g.ldhc + col0 + i] =
-                    __float2bfloat16_rn(x);
             }
           }
         }
+        __syncwarp();
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&tl->acc_empty[acc]);
+      if (lane == 0) mbar_arrive_cluster(acc_empty0[acc]);
+    }
+  } else {
+    // ------------------------------------------------ residual epilogue (warps 2..5, both CTAs)
+    // h += C for this warp's 32 rows, 32 columns at a time: TMA brings the h
+    // chunk into a 128-byte-swizzled slot (prefetched two chunks ahead), the
+    // thread owning a row adds its accumulator row in place (the swizzle keeps
+    // the row-per-thread access free of bank conflicts), and TMA writes h and
+    // its bf16 copy back.
+    const int q = warp & 3;
+    uint8_t* wbuf = smem + Layout<EPI>::EPI_OFF + q * RES_WARP_BYTES;
+    uint64_t* hbar = tl->hbar[q];
+    const uint32_t acc_empty0[2] = {cluster_map(&tl->acc_empty[0], 0),
+                                    cluster_map(&tl->acc_empty[1], 0)};
+    const bool copy = g.h_copy != nullptr;
+    uint32_t hph[2] = {0u, 0u};
+    bool pending[2] = {false, false};
+    bool ok = true;
+    int local = 0;
+    for (int tile = cluster; tile < num_tiles && ok; tile += n_clusters, ++local) {
+      const int acc = local & 1;
+      const uint32_t acc_phase = (local >> 1) & 1;
+      int m_blk, n_blk;
+      tile_coords(tile, m_tiles, n_tiles, group, m_blk, n_blk);
+      const int64_t row0 = static_cast<int64_t>(m_blk) * BM + rank * HALF + q * 32;
+      const int64_t colT = static_cast<int64_t>(n_blk) * BN;
+      const int64_t left = (g.N - colT + 31) / 32;
+      const int nch = row0 < g.M ? static_cast<int>(left < 8 ? left : 8) : 0;
+      if (lane == 0) {
+        tma_store_wait_read0();  // both slots free again
+        for (int c = 0; c < min(2, nch); ++c) {
+          mbar_arrive_expect_tx(&hbar[c], RES_H_BYTES);
+          tma_load_2d(&map_h, &hbar[c], wbuf + c * RES_H_BYTES, static_cast<int>(colT + 32 * c),
+                      static_cast<int>(row0));
+          pending[c] = true;
+        }
+      }
+      const bool w = mbar_wait(&tl->acc_full[acc], acc_phase, abort_flag, g.status, WHERE_GEMM);
+      if (!__all_sync(0xffffffffu, w)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+#pragma unroll 1
+      for (int c = 0; c < nch; ++c) {
+        uint32_t r[32];
+        tmem_ld32(tmem_base + (static_cast<uint32_t>(q * 32) << 16) + acc * BN + 32 * c, r);
+        tmem_wait_ld();
+        const int sl = c & 1;
+        const bool wh = mbar_wait(&hbar[sl], hph[sl], abort_flag, g.status, WHERE_GEMM);
+        if (!__all_sync(0xffffffffu, wh)) {
+          ok = false;
+          break;
+        }
+        hph[sl] ^= 1u;
+        pending[sl] = false;
+        float* hs = reinterpret_cast<float*>(wbuf + sl * RES_H_BYTES);
+        uint8_t* cs = wbuf + 2 * RES_H_BYTES + sl * RES_C_BYTES;
+        float hv[32];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          float4* a = reinterpret_cast<float4*>(hs + lane * 32 + 4 * (k ^ (lane & 7)));
+          float4 x = *a;
+          x.x += __uint_as_float(r[4 * k]);
+          x.y += __uint_as_float(r[4 * k + 1]);
+          x.z += __uint_as_float(r[4 * k + 2]);
+          x.w += __uint_as_float(r[4 * k + 3]);
+          *a = x;
+          hv[4 * k] = x.x; hv[4 * k + 1] = x.y; hv[4 * k + 2] = x.z; hv[4 * k + 3] = x.w;
+        }
+        if (copy) {
+#pragma unroll
+          for (int k = 0; k < 4; ++k)
+            *reinterpret_cast<uint4*>(cs + lane * 64 + 16 * (k ^ ((lane >> 1) & 3))) =
+                make_uint4(pack_bf16x2(hv[8 * k], hv[8 * k + 1]), pack_bf16x2(hv[8 * k + 2], hv[8 * k + 3]),
+                           pack_bf16x2(hv[8 * k + 4], hv[8 * k + 5]), pack_bf16x2(hv[8 * k + 6], hv[8 * k + 7]));
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          const int x = static_cast<int>(colT + 32 * c), y = static_cast<int>(row0);
+          tma_store_2d(&map_h, hs, x, y);
+          if (copy) tma_store_2d(&map_c, cs, x, y);
+          tma_store_commit();
+          if (c + 2 < nch) {
+            tma_store_wait_read0();  // the slot's stores have read it
+            mbar_arrive_expect_tx(&hbar[sl], RES_H_BYTES);
+            tma_load_2d(&map_h, &hbar[sl], hs, x + 64, y);
+            pending[sl] = true;
+          }
+        }
+        __syncwarp();
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(acc_empty0[acc]);
+    }
+    if (lane == 0) {
+      for (int sl = 0; sl < 2; ++sl)
+        if (pending[sl]) (void)drain_wait(&hbar[sl], hph[sl]);
+      tma_store_wait0();
     }
   }
 
   tc_fence_before();
   __syncthreads();
+  cluster_sync();  // neither CTA leaves while the pair's MMAs may still read its tiles
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem_base, TMEM_COLS);
+    tmem_dealloc_pair(tmem_base, TMEM_COLS);
   }
+}
+
+template <int EPI>
+cudaError_t launch(const CUtensorMap& ma, const CUtensorMap& mb, const CUtensorMap& mh,
+                   const CUtensorMap& mc, const GemmArgs& g, int grid, int group, cudaStream_t s) {
+  auto kern = gemm_bf16_tc_kernel<EPI>;
+  constexpr size_t kGemmSmem = gemm_smem<EPI>();
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(kGemmSmem));
+  if (e != cudaSuccess) return e;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid, 1, 1);
+  cfg.blockDim = dim3(NUM_THREADS, 1, 1);
+  cfg.dynamicSmemBytes = kGemmSmem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, ma, mb, mh, mc, g, group);
 }
 
 }  // namespace
@@ -261,7 +414,7 @@ cudaError_t gemm_bf16(const GemmArgs& g, cudaStream_t s) {
   {
     const uint64_t dims[2] = {static_cast<uint64_t>(g.K), static_cast<uint64_t>(g.M)};
     const uint64_t strides[1] = {static_cast<uint64_t>(g.lda) * 2};
-    const uint32_t box[2] = {BK, BM};
+    const uint32_t box[2] = {BK, HALF};
     if (!encode_tmap(&ma, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, g.a, dims, strides, box,
                      CU_TENSOR_MAP_SWIZZLE_128B))
       return cudaErrorInvalidValue;
@@ -269,26 +422,40 @@ cudaError_t gemm_bf16(const GemmArgs& g, cudaStream_t s) {
   {
     const uint64_t dims[2] = {static_cast<uint64_t>(g.K), static_cast<uint64_t>(g.N)};
     const uint64_t strides[1] = {static_cast<uint64_t>(g.ldb) * 2};
-    const uint32_t box[2] = {BK, BN};
+    const uint32_t box[2] = {BK, HALF};
     if (!encode_tmap(&mb, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, g.b, dims, strides, box,
                      CU_TENSOR_MAP_SWIZZLE_128B))
       return cudaErrorInvalidValue;
   }
-  const int64_t tiles = ((g.M + BM - 1) / BM) * ((g.N + BN - 1) / BN);
-  const int grid = static_cast<int>(std::min<int64_t>(tiles, device_sm_count()));
-  cudaError_t e;
-  if (g.epi == EPI_STORE) {
-    e = cudaFuncSetAttribute(gemm_bf16_tc_kernel<EPI_STORE>,
-                             cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(kGemmSmem));
-    if (e != cudaSuccess) return e;
-    gemm_bf16_tc_kernel<EPI_STORE><<<grid, NUM_THREADS, kGemmSmem, s>>>(ma, mb, g);
-  } else {
-    e = cudaFuncSetAttribute(gemm_bf16_tc_kernel<EPI_RESIDUAL>,
-                             cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(kGemmSmem));
-    if (e != cudaSuccess) return e;
-    gemm_bf16_tc_kernel<EPI_RESIDUAL><<<grid, NUM_THREADS, kGemmSmem, s>>>(ma, mb, g);
+  const int64_t m_tiles = (g.M + BM - 1) / BM, n_tiles = (g.N + BN - 1) / BN;
+  const int64_t tiles = m_tiles * n_tiles;
+  const int clusters = static_cast<int>(std::max<int64_t>(
+      1, std::min<int64_t>(tiles, device_sm_count() / 2)));
+  // a wave of clusters covers `group` M tiles by about four N tiles
+  const int group = static_cast<int>(std::max<int64_t>(
+      1, std::min<int64_t>(m_tiles, clusters / std::min<int64_t>(4, n_tiles))));
+  if (g.epi == EPI_STORE) return launch<EPI_STORE>(ma, mb, ma, ma, g, 2 * clusters, group, s);
+  // residual epilogue: h (fp32, 32x32 boxes, 128-byte swizzle) and its bf16
+  // copy (32x32 boxes, 64-byte swizzle); without a copy the h map stands in
+  CUtensorMap mh, mc;
+  {
+    const uint64_t dims[2] = {static_cast<uint64_t>(g.N), static_cast<uint64_t>(g.M)};
+    const uint64_t strides[1] = {static_cast<uint64_t>(g.ldh) * 4};
+    const uint32_t box[2] = {32, 32};
+    if (!encode_tmap(&mh, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, g.h, dims, strides, box,
+                     CU_TENSOR_MAP_SWIZZLE_128B))
+      return cudaErrorInvalidValue;
   }
-  return cudaGetLastError();
+  mc = mh;
+  if (g.h_copy != nullptr) {
+    const uint64_t dims[2] = {static_cast<uint64_t>(g.N), static_cast<uint64_t>(g.M)};
+    const uint64_t strides[1] = {static_cast<uint64_t>(g.ldhc) * 2};
+    const uint32_t box[2] = {32, 32};
+    if (!encode_tmap(&mc, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, g.h_copy, dims, strides, box,
+                     CU_TENSOR_MAP_SWIZZLE_64B))
+      return cudaErrorInvalidValue;
+  }
+  return launch<EPI_RESIDUAL>(ma, mb, mh, mc, g, 2 * clusters, group, s);
 }
 
 }  // namespace sva

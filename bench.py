@@ -59,6 +59,28 @@ def load_peaks():
     return dict(FALLBACK_PEAKS, source="fallback")
 
 
+def profiled_traffic(kind: str):
+    """DRAM bytes per launch of a kernel class from the committed ncu capture
+    (profiles/traffic.json), or None when the kernel's source has changed since
+    (its hash no longer matches) or no capture exists."""
+    import hashlib
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(path):
+        return None, None
+    with open(path) as f:
+        entry = json.load(f).get(kind)
+    if entry is None:
+        return None, None
+    csrc = os.path.join(ROOT, "softmax_attention_video_gated_b200", "csrc")
+    h = hashlib.sha256()
+    for name in (entry["source"], "common.cuh"):
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(f.read())
+    if h.hexdigest()[:16] != entry["source_hash"]:
+        return None, None
+    return entry["bytes_per_launch"], entry["profile"]
+
+
 def algorithmic_work(kind: str, wl: dict, n_blocks_routed: int = 1):
     """Algorithmic FLOPs or bytes of one launch of a kernel class.
 
@@ -485,16 +507,21 @@ def main():
     dom = max((k for k in kernels if k != "other"), key=lambda k: kernels[k]["ms_per_step"])
     bound, work = algorithmic_work(dom, wl, 1)
     de = kernels[dom]
+    traffic, traffic_src = profiled_traffic(dom)
     if bound == "tensor":
         roof = {"kernel": dom, "bound": "tensor", "achieved": de["achieved"],
                 "peak": peaks["bf16_tflops_sustained"], "unit": "TFLOP/s",
                 "frac": de["achieved"] / peaks["bf16_tflops_sustained"],
                 "peak_source": f"{peaks['source']} bf16_tflops_sustained (kernel timed inside a long step)",
-                "traffic": None}
+                "traffic": traffic}
     else:
         roof = {"kernel": dom, "bound": "hbm", "achieved": de["achieved"], "peak": peaks["hbm_gbs"],
                 "unit": "GB/s", "frac": de["achieved"] / peaks["hbm_gbs"],
-                "peak_source": f"{peaks['source']} hbm_gbs", "traffic": None}
+                "peak_source": f"{peaks['source']} hbm_gbs", "traffic": traffic}
+    roof["algorithmic_per_launch"] = work
+    if traffic is not None:
+        roof["traffic_unit"] = "bytes per launch (dram read + write)"
+        roof["traffic_source"] = traffic_src
 
     # ---- end to end through the C ABI: pinned host input in, result read back
     xh = x.cpu().pin_memory()

@@ -88,10 +88,11 @@ def lin_state(k: np.ndarray, v: np.ndarray, H: int) -> Tuple[np.ndarray, np.ndar
     """State of every (batch, head) over all N tokens.
 
     S[b, h] = sum_t phi(K_t)^T V_t   (d x d),   z[b, h] = sum_t phi(K_t)   (d).
-    Returns S [B, H, d, d] and z [B, H, d]."""
+    Returns S [B, H, d, d] and z [B, H, d]. (The sum over tokens is a plain
+    matrix product phi(K)^T V.)"""
     fk = phi(split_heads(k, H))
     vh = split_heads(v, H)
-    S = np.einsum("bhtk,bhtv->bhkv", fk, vh)
+    S = np.matmul(np.swapaxes(fk, -1, -2), vh)
     z = fk.sum(axis=2)
     return S, z
 
@@ -101,8 +102,8 @@ def lin_readout(q: np.ndarray, S: np.ndarray, z: np.ndarray, H: int, eps: float)
 
     q may hold any subset of rows; S and z come from `lin_state`."""
     fq = phi(split_heads(q, H))
-    num = np.einsum("bhtk,bhkv->bhtv", fq, S)
-    den = np.einsum("bhtk,bhk->bht", fq, z) + eps
+    num = np.matmul(fq, S)
+    den = np.matmul(fq, z[..., None])[..., 0] + eps
     return merge_heads(num / den[..., None])
 
 

@@ -7,7 +7,10 @@
 //
 // One CTA per pair of 128-query tiles of one (head, batch); 12 warps in three
 // warpgroups:
-//   WG0  warp 0: TMA (both Q tiles once, then 128-key K and V tiles, 2 stages);
+//   WG0  warp 0: TMA for both Q tiles once, then the 128-key K tiles (3-stage
+//        ring); warp 2: TMA for the V tiles (2-stage ring). K is released as
+//        soon as both S MMAs of a block have read it, V after both P V MMAs,
+//        so the next block's K is already resident when its S MMA is due.
 //        warp 1: allocates all 512 TMEM columns (tile t: S_t at 256t, O_t at
 //        256t+128) and issues every MMA from one thread. Registers shrink to 56.
 //   WG1, WG2  softmax of tile 0 and tile 1: thread r owns query row r (its
@@ -21,9 +24,12 @@
 // that sees S_{j+1} may rescale O.
 // Softmax per row: running max in the log2 domain, rescaled only when it grows
 // by more than 8 (p <= 2^8 otherwise, exact after the final 1/l); one FFMA per
-// element folds the scale; three of every four exponentials go to the MUFU
-// unit and one to the FMA pipe (Cody-Waite reduction and a minimax cubic, see
-// fit_exp2_poly.py), which takes load off the MUFU unit.
+// element folds the scale. Exponentials run on the MUFU unit; kPolyEvery can
+// send every k-th one to the FMA pipe instead (Cody-Waite reduction and a
+// minimax cubic, see fit_exp2_poly.py). Measured on B200 at 720p: all-MUFU
+// 4.37 ms, one in four on the FMA pipe 4.77 ms, one in two 5.26 ms, and no
+// exponentials at all 4.26 ms -- this kernel is bound by its MMA pipeline
+// (3.54 ms with an empty softmax), not by the exponentials.
 #include <algorithm>
 #include <math.h>
 
@@ -36,26 +42,29 @@ namespace {
 constexpr int HD = 128;
 constexpr int BQ = 128, BKV = 128;
 constexpr int BOX = 128 * 128;              // [64 cols x 128 rows] bf16 = 16 KB
-constexpr int KV_STAGES = 2;
+constexpr int K_STAGES = 3, V_STAGES = 2;
 constexpr int Q_OFF = 0;                     // tile t: 32 KB at Q_OFF + t * 2 * BOX
-constexpr int KV_OFF = 4 * BOX;              // stage s: K at +s*64K, V at +s*64K+32K
-constexpr int KV_STAGE_BYTES = 4 * BOX;
-constexpr int TAIL_OFF = KV_OFF + KV_STAGES * KV_STAGE_BYTES;
+constexpr int K_OFF = 4 * BOX;               // K stage s: 32 KB at K_OFF + s * 2 * BOX
+constexpr int V_OFF = K_OFF + K_STAGES * 2 * BOX;
+constexpr int TAIL_OFF = V_OFF + V_STAGES * 2 * BOX;
 constexpr int NUM_THREADS = 384;
 constexpr int TMEM_COLS = 512;
 constexpr float kRescaleThreshold = 8.0f;    // log2 units
 // register split: 128 threads at 56 + 256 threads at 224 = 384 threads at 168
 constexpr int kRegsProducer = 56, kRegsSoftmax = 224;
 
+// every kPolyEvery-th exponential of a row is evaluated on the FMA pipe (0: none)
+constexpr int kPolyEvery = 0;
 // minimax cubic for 2^f on [-1/2, 1/2] with c0 = 1 (fit_exp2_poly.py);
 // max relative error 4.4e-4, five times below bf16's rounding of P
 constexpr float kP1 = 0.695766806602478f, kP2 = 0.24203051626682281f, kP3 = 0.041698750108480453f;
 
 struct AnchorTail {
   uint64_t q_full;
-  uint64_t k_full[KV_STAGES];
-  uint64_t v_full[KV_STAGES];
-  uint64_t kv_empty[KV_STAGES];
+  uint64_t k_full[K_STAGES];
+  uint64_t k_empty[K_STAGES];
+  uint64_t v_full[V_STAGES];
+  uint64_t v_empty[V_STAGES];
   uint64_t s_full[2];
   uint64_t p_full[2];
   uint64_t o_done;
@@ -106,10 +115,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 
   if (threadIdx.x == 0) {
     mbar_init(&tl->q_full, 1);
-    for (int s = 0; s < KV_STAGES; ++s) {
+    for (int s = 0; s < K_STAGES; ++s) {
       mbar_init(&tl->k_full[s], 1);
+      mbar_init(&tl->k_empty[s], 1);
+    }
+    for (int s = 0; s < V_STAGES; ++s) {
       mbar_init(&tl->v_full[s], 1);
-      mbar_init(&tl->kv_empty[s], 1);
+      mbar_init(&tl->v_empty[s], 1);
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&tl->s_full[i], 1);
@@ -138,7 +150,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   if (wg == 0) {
     warpgroup_reg_dec<kRegsProducer>();
     if (warp == 0 && lane == 0) {
-      // ------------------------------------------------ TMA producer
+      // ------------------------------------------------ TMA producer: Q, then K
       mbar_arrive_expect_tx(&tl->q_full, (has1 ? 4 : 2) * BOX);
       tma_load_3d(&map_q, &tl->q_full, smem + Q_OFF, h * HD, q0, b);
       tma_load_3d(&map_q, &tl->q_full, smem + Q_OFF + BOX, h * HD + 64, q0, b);
@@ -149,27 +161,42 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       int issued = 0;
       bool ok = true;
       for (int j = 0; j < nkv; ++j) {
-        const int st = j % KV_STAGES;
-        const uint32_t ph = (j / KV_STAGES) & 1;
-        if (!mbar_wait(&tl->kv_empty[st], ph ^ 1, abort_flag, status, WHERE_ANCHOR)) {
+        const int st = j % K_STAGES;
+        if (!mbar_wait(&tl->k_empty[st], ((j / K_STAGES) & 1) ^ 1, abort_flag, status,
+                       WHERE_ANCHOR)) {
           ok = false;
           break;
         }
-        uint8_t* kt = smem + KV_OFF + st * KV_STAGE_BYTES;
+        uint8_t* kt = smem + K_OFF + st * 2 * BOX;
         mbar_arrive_expect_tx(&tl->k_full[st], 2 * BOX);
         tma_load_3d(&map_k, &tl->k_full[st], kt, h * HD, j * BKV, b);
         tma_load_3d(&map_k, &tl->k_full[st], kt + BOX, h * HD + 64, j * BKV, b);
-        mbar_arrive_expect_tx(&tl->v_full[st], 2 * BOX);
-        tma_load_3d(&map_v, &tl->v_full[st], kt + 2 * BOX, h * HD, j * BKV, b);
-        tma_load_3d(&map_v, &tl->v_full[st], kt + 3 * BOX, h * HD + 64, j * BKV, b);
         ++issued;
       }
       (void)drain_wait(&tl->q_full, 0);
       if (!ok)
-        for (int i = max(0, issued - KV_STAGES); i < issued; ++i) {
-          (void)drain_wait(&tl->k_full[i % KV_STAGES], (i / KV_STAGES) & 1);
-          (void)drain_wait(&tl->v_full[i % KV_STAGES], (i / KV_STAGES) & 1);
+        for (int i = max(0, issued - K_STAGES); i < issued; ++i)
+          (void)drain_wait(&tl->k_full[i % K_STAGES], (i / K_STAGES) & 1);
+    } else if (warp == 2 && lane == 0) {
+      // ------------------------------------------------ TMA producer: V
+      int issued = 0;
+      bool ok = true;
+      for (int j = 0; j < nkv; ++j) {
+        const int st = j % V_STAGES;
+        if (!mbar_wait(&tl->v_empty[st], ((j / V_STAGES) & 1) ^ 1, abort_flag, status,
+                       WHERE_ANCHOR)) {
+          ok = false;
+          break;
         }
+        uint8_t* vt = smem + V_OFF + st * 2 * BOX;
+        mbar_arrive_expect_tx(&tl->v_full[st], 2 * BOX);
+        tma_load_3d(&map_v, &tl->v_full[st], vt, h * HD, j * BKV, b);
+        tma_load_3d(&map_v, &tl->v_full[st], vt + BOX, h * HD + 64, j * BKV, b);
+        ++issued;
+      }
+      if (!ok)
+        for (int i = max(0, issued - V_STAGES); i < issued; ++i)
+          (void)drain_wait(&tl->v_full[i % V_STAGES], (i / V_STAGES) & 1);
     } else if (warp == 1 && lane == 0) {
       // ------------------------------------------------ MMA issuer
       constexpr uint32_t idesc_s = idesc_bf16_f32(BQ, BKV, false, false);  // Q, K: K-major
@@ -178,7 +205,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       bool ok = mbar_wait(&tl->q_full, 0, abort_flag, status, WHERE_ANCHOR);
       auto issue_s = [&](int t, int j) {
         const uint32_t qaddr = smem_u32(smem + Q_OFF + t * 2 * BOX);
-        const uint32_t kaddr = smem_u32(smem + KV_OFF + (j % KV_STAGES) * KV_STAGE_BYTES);
+        const uint32_t kaddr = smem_u32(smem + K_OFF + (j % K_STAGES) * 2 * BOX);
         const uint32_t d_tmem = tmem + t * 256;
 #pragma unroll
         for (int kk = 0; kk < HD / 16; ++kk) {
@@ -190,8 +217,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         umma_commit(&tl->s_full[t]);
       };
       auto issue_pv = [&](int t, int j) {
-        const uint32_t vaddr =
-            smem_u32(smem + KV_OFF + (j % KV_STAGES) * KV_STAGE_BYTES + 2 * BOX);
+        const uint32_t vaddr = smem_u32(smem + V_OFF + (j % V_STAGES) * 2 * BOX);
         const uint32_t p_tmem = tmem + t * 256;
 #pragma unroll
         for (int kk = 0; kk < BKV / 16; ++kk) {
@@ -204,14 +230,16 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         if (ok) {
           tc_fence_after();
           for (int t = 0; t < ntiles; ++t) issue_s(t, 0);
+          umma_commit(&tl->k_empty[0]);
         }
       }
       for (int j = 0; j < nkv && ok; ++j) {
-        const int st = j % KV_STAGES;
         const bool more = j + 1 < nkv;
-        if (!mbar_wait(&tl->v_full[st], (j / KV_STAGES) & 1, abort_flag, status, WHERE_ANCHOR) ||
-            (more && !mbar_wait(&tl->k_full[(j + 1) % KV_STAGES], ((j + 1) / KV_STAGES) & 1,
-                                abort_flag, status, WHERE_ANCHOR))) {
+        const int kn = (j + 1) % K_STAGES;
+        if (!mbar_wait(&tl->v_full[j % V_STAGES], (j / V_STAGES) & 1, abort_flag, status,
+                       WHERE_ANCHOR) ||
+            (more && !mbar_wait(&tl->k_full[kn], ((j + 1) / K_STAGES) & 1, abort_flag, status,
+                                WHERE_ANCHOR))) {
           ok = false;
           break;
         }
@@ -222,8 +250,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           }
           tc_fence_after();
           issue_pv(t, j);
-          if (t == ntiles - 1) umma_commit(&tl->kv_empty[st]);
-          if (more) issue_s(t, j + 1);
+          if (t == ntiles - 1) umma_commit(&tl->v_empty[j % V_STAGES]);
+          if (more) {
+            issue_s(t, j + 1);
+            if (t == ntiles - 1) umma_commit(&tl->k_empty[kn]);
+          }
         }
       }
       if (ok) umma_commit(&tl->o_done);
@@ -305,7 +336,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             const float x0 = fmaf(s[32 * c + 2 * i], scale_log2, neg_m);
             const float x1 = fmaf(s[32 * c + 2 * i + 1], scale_log2, neg_m);
             const float p0 = ex2_mufu(x0);
-            const float p1 = (i & 1) ? ex2_poly(x1) : ex2_mufu(x1);  // 1 in 4 on the FMA pipe
+            const float p1 = (kPolyEvery > 0 && (2 * i + 1) % kPolyEvery == kPolyEvery - 1)
+                                 ? ex2_poly(x1)
+                                 : ex2_mufu(x1);
             acc[i & 7] += p0 + p1;
             pk[i] = pack_bf16x2(p0, p1);
           }

@@ -136,6 +136,39 @@ def normal(shape, std: float, seed: int, tag: int, dtype: str) -> np.ndarray:
     return round_to(a, dtype)
 
 
+def normal_par(shape, std: float, seed: int, tag: int, dtype: str, rows_per_chunk: int = 4096,
+               threads: int = 0) -> np.ndarray:
+    """N(0, std^2) like `normal`, for large tensors: the leading-axis-flattened
+    rows are drawn in chunks of `rows_per_chunk`, chunk i from its own stream
+    SeedSequence([seed, tag, i]), on a thread pool. The values depend only on
+    (shape, seed, tag, rows_per_chunk), not on the number of threads."""
+    import concurrent.futures as cf
+    import os
+    shape = tuple(shape)
+    rows = int(np.prod(shape[:-1])) if len(shape) > 1 else 1
+    width = shape[-1]
+    out = np.empty((rows, width), dtype=np.float32)
+
+    def fill(i):
+        r0, r1 = i * rows_per_chunk, min(rows, (i + 1) * rows_per_chunk)
+        g = np.random.Generator(np.random.PCG64(np.random.SeedSequence([seed, tag, i])))
+        a = g.standard_normal(size=(r1 - r0, width), dtype=np.float32)
+        if std != 1.0:
+            a *= np.float32(std)
+        out[r0:r1] = round_to(a, dtype)
+
+    n = (rows + rows_per_chunk - 1) // rows_per_chunk
+    with cf.ThreadPoolExecutor(threads or min(32, os.cpu_count() or 1)) as ex:
+        list(ex.map(fill, range(n)))
+    return out.reshape(shape)
+
+
+def core_inputs_par(B: int, N: int, H: int, d: int, dtype: str, seed: int) -> Dict[str, np.ndarray]:
+    """Q, K, V, G ~ N(0, 1) of [B, N, H*d] drawn with `normal_par`."""
+    return {name: normal_par((B, N, H * d), 1.0, seed, tag, dtype)
+            for name, tag in (("q", TAG_Q), ("k", TAG_K), ("v", TAG_V), ("g", TAG_G))}
+
+
 def core_inputs(B: int, N: int, H: int, d: int, dtype: str, seed: int,
                 q_scale: float = 1.0) -> Dict[str, np.ndarray]:
     """Q, K, V, gate logits G ~ N(0, 1), each [B, N, H*d]. `q_scale` scales Q

@@ -170,6 +170,22 @@ def gpu_uuid(torch, dev):
         return None
 
 
+def max_over_ranks(v: float, dist=None, device="cpu") -> float:
+    """The maximum of a per-rank value over all ranks (a no-op on one rank)."""
+    if dist is None or not dist.is_initialized() or dist.get_world_size() == 1:
+        return v
+    import torch
+    t = torch.tensor([v], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_rate(world: int, tokens_per_rank: int, ms_per_step: float) -> float:
+    """Tokens per second of the whole job: every rank runs its own replica of the
+    stack on its own tokens, and the slowest rank sets the step time."""
+    return world * tokens_per_rank / (ms_per_step * 1e-3)
+
+
 def blas_threads():
     try:
         from threadpoolctl import threadpool_info
@@ -475,13 +491,6 @@ def main():
         if dist is not None:
             dist.barrier()
 
-    def max_over_ranks(v):
-        if dist is None:
-            return v
-        t = torch.tensor([v], dtype=torch.float64, device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
-
     for _ in range(args.warmup):
         sva.sva_hybrid_stack_fwd(stack, x, y, ws)
     st = sva.sva_check_device_status(ws)
@@ -500,8 +509,8 @@ def main():
     st = sva.sva_check_device_status(ws)
     if st != sva.SVA_OK:
         raise RuntimeError(f"device status after the timed region: {sva.status_string(st)}")
-    ms_step = max_over_ranks(ms_total / args.steps)
-    value = world * B * N / (ms_step * 1e-3)
+    ms_step = max_over_ranks(ms_total / args.steps, dist, "cuda")
+    value = whole_job_rate(world, B * N, ms_step)
 
     kernels = summarize(recs, args.steps, wl, peaks)
     dom = max((k for k in kernels if k != "other"), key=lambda k: kernels[k]["ms_per_step"])
@@ -541,7 +550,7 @@ def main():
         yh.copy_(y, non_blocking=True)
     e1.record()
     torch.cuda.synchronize()
-    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / args.steps)
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / args.steps, dist, "cuda")
     barrier()
 
     # ---- the all-softmax stack of the same shape (quadratic baseline)
@@ -566,7 +575,7 @@ def main():
         "data": "synthetic (seeded: x ~ N(0,1), weights ~ N(0,1/D))",
         "config": config_block(wl, world),
         "roofline": roof,
-        "e2e": {"value": world * B * N / (e2e_ms * 1e-3), "unit": "tokens/s",
+        "e2e": {"value": whole_job_rate(world, B * N, e2e_ms), "unit": "tokens/s",
                 "h2d_bytes_per_step": xh.numel() * xh.element_size(),
                 "d2h_bytes_per_step": yh.numel() * yh.element_size()},
         "gpu_launches": launches,

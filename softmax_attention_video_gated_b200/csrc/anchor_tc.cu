@@ -97,6 +97,15 @@ __device__ __forceinline__ float ex2_poly(float x) {
   return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
 }
 
+// exponential of the element at position `idx` of a row
+template <int kEvery>
+__device__ __forceinline__ float ex2_row(float x, int idx) {
+  if constexpr (kEvery > 0) {
+    if (idx % kEvery == kEvery - 1) return ex2_poly(x);
+  }
+  return ex2_mufu(x);
+}
+
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     anchor_tc_kernel(const __grid_constant__ CUtensorMap map_q,
                      const __grid_constant__ CUtensorMap map_k,
@@ -335,10 +344,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           for (int i = 0; i < 16; ++i) {
             const float x0 = fmaf(s[32 * c + 2 * i], scale_log2, neg_m);
             const float x1 = fmaf(s[32 * c + 2 * i + 1], scale_log2, neg_m);
-            const float p0 = ex2_mufu(x0);
-            const float p1 = (kPolyEvery > 0 && (2 * i + 1) % kPolyEvery == kPolyEvery - 1)
-                                 ? ex2_poly(x1)
-                                 : ex2_mufu(x1);
+            const float p0 = ex2_row<kPolyEvery>(x0, 2 * i);
+            const float p1 = ex2_row<kPolyEvery>(x1, 2 * i + 1);
             acc[i & 7] += p0 + p1;
             pk[i] = pack_bf16x2(p0, p1);
           }

@@ -29,6 +29,9 @@ are silent (each is marked "reading"):
   A_t = phi(Q_t) S / (phi(Q_t) . z + eps)               (non-causal, reading)
   A_t = sum_s softmax_s(Q_t . K_s / sqrt(d)) V_s         (non-causal)
   Y = A * sigmoid(G)                                     (per-channel output gate, reading)
+  write-gated variant: token t's write into the state of head h is scaled by
+     omega_t = sigmoid(W_t) (one logit per token and head, W = u W_w^T):
+     S = sum_t omega_t phi(K_t)^T V_t,  z = sum_t omega_t phi(K_t)      (reading)
   [Q | K | V | G] = u W_qkvg^T,  o = Y W_o^T,  h_l = h_{l-1} + o
   router (linear layers of block c >= 2):
      q = h_{l-1} W_r^T
@@ -49,7 +52,7 @@ from typing import Dict, List, Optional, Sequence, Tuple
 import numpy as np
 
 __all__ = [
-    "phi", "split_heads", "merge_heads", "lin_state", "lin_readout", "lin_core",
+    "phi", "split_heads", "merge_heads", "write_weights", "lin_state", "lin_readout", "lin_core",
     "lin_core_bruteforce", "softmax_core", "sigmoid", "gate", "linear_attn",
     "softmax_anchor", "project", "route", "layer_kind", "block_of", "stack",
 ]
@@ -84,13 +87,29 @@ def merge_heads(a: np.ndarray) -> np.ndarray:
 # ---------------------------------------------------------------------------
 
 
-def lin_state(k: np.ndarray, v: np.ndarray, H: int) -> Tuple[np.ndarray, np.ndarray]:
+def write_weights(wgate, H: int) -> np.ndarray:
+    """omega [B, H, N, 1] = sigmoid of the write-gate logits [B, N, H].
+
+    The gate sets how much each token writes into the fixed-size state
+    [ai-papers.net summary, section "ハイブリッド線形アテンション"]; the reading
+    taken here is one logit per token and head, scaling that token's whole
+    write (its term in S and in z)."""
+    w = _f64(wgate)
+    assert w.ndim == 3 and w.shape[2] == H
+    return sigmoid(w).transpose(0, 2, 1)[..., None]
+
+
+def lin_state(k: np.ndarray, v: np.ndarray, H: int, wgate=None) -> Tuple[np.ndarray, np.ndarray]:
     """State of every (batch, head) over all N tokens.
 
     S[b, h] = sum_t phi(K_t)^T V_t   (d x d),   z[b, h] = sum_t phi(K_t)   (d).
+    With write-gate logits wgate [B, N, H] every token's term is scaled by
+    omega_t = sigmoid(wgate[b, t, h]) in both sums.
     Returns S [B, H, d, d] and z [B, H, d]. (The sum over tokens is a plain
     matrix product phi(K)^T V.)"""
     fk = phi(split_heads(k, H))
+    if wgate is not None:
+        fk = fk * write_weights(wgate, H)
     vh = split_heads(v, H)
     S = np.matmul(np.swapaxes(fk, -1, -2), vh)
     z = fk.sum(axis=2)
@@ -107,23 +126,27 @@ def lin_readout(q: np.ndarray, S: np.ndarray, z: np.ndarray, H: int, eps: float)
     return merge_heads(num / den[..., None])
 
 
-def lin_core(q, k, v, H: int, eps: float = 1e-6) -> np.ndarray:
+def lin_core(q, k, v, H: int, eps: float = 1e-6, wgate=None) -> np.ndarray:
     """Normalised non-causal linear attention, associative (state) form."""
-    S, z = lin_state(k, v, H)
+    S, z = lin_state(k, v, H, wgate)
     return lin_readout(q, S, z, H, eps)
 
 
-def lin_core_bruteforce(q, k, v, H: int, eps: float = 1e-6) -> np.ndarray:
+def lin_core_bruteforce(q, k, v, H: int, eps: float = 1e-6, wgate=None) -> np.ndarray:
     """The same quantity in its O(N^2) pairwise form, with an explicit loop over
-    query tokens: A_t = sum_s w_ts V_s / (sum_s w_ts + eps), w_ts = phi(Q_t).phi(K_s).
+    query tokens: A_t = sum_s w_ts V_s / (sum_s w_ts + eps), w_ts = phi(Q_t).phi(K_s),
+    times omega_s = sigmoid(wgate[b, s, h]) when write-gate logits are given.
     Used only to pin `lin_core` on small N."""
     fq, fk, vh = phi(split_heads(q, H)), phi(split_heads(k, H)), split_heads(v, H)
     B, _, Nq, d = fq.shape
+    Nk = fk.shape[2]
     out = np.zeros((B, H, Nq, vh.shape[-1]))
     for b in range(B):
         for h in range(H):
+            om = np.ones(Nk) if wgate is None else np.array(
+                [1.0 / (1.0 + math.exp(-float(wgate[b, s, h]))) for s in range(Nk)])
             for t in range(Nq):
-                w = fk[b, h] @ fq[b, h, t]              # w_ts for all s
+                w = (fk[b, h] @ fq[b, h, t]) * om       # w_ts for all s
                 out[b, h, t] = (w @ vh[b, h]) / (w.sum() + eps)
     return merge_heads(out)
 
@@ -173,9 +196,10 @@ def gate(a, g) -> np.ndarray:
     return _f64(a) * sigmoid(g)
 
 
-def linear_attn(q, k, v, g, H: int, eps: float = 1e-6, residual=None) -> np.ndarray:
-    """Gated linear-attention layer core: Y = lin_core(Q, K, V) * sigmoid(G) (+ residual)."""
-    y = gate(lin_core(q, k, v, H, eps), g)
+def linear_attn(q, k, v, g, H: int, eps: float = 1e-6, residual=None, wgate=None) -> np.ndarray:
+    """Gated linear-attention layer core: Y = lin_core(Q, K, V) * sigmoid(G) (+ residual);
+    wgate [B, N, H] (optional) are the write-gate logits of the state."""
+    y = gate(lin_core(q, k, v, H, eps, wgate), g)
     return y if residual is None else y + _f64(residual)
 
 
@@ -236,13 +260,15 @@ def block_of(l: int, attnres_block: int) -> int:
 
 def stack(x, w_qkvg: Sequence[np.ndarray], w_o: Sequence[np.ndarray], w_r, H: int,
           softmax_period: int = 4, attnres_block: int = 8, all_softmax: bool = False,
-          eps: float = 1e-6, keep_trace: bool = False):
+          eps: float = 1e-6, keep_trace: bool = False, w_wg: Optional[Sequence] = None):
     """The hybrid token mixer: tokens in, mixed tokens out.
 
     h_0 = x; for l = 1..L: u = routed or plain input, [Q|K|V|G] = u W_qkvg[l]^T,
     Y = gated linear or softmax core, h_l = h_{l-1} + Y W_o[l]^T.
     Summaries s_c = h_{8c} are kept after each completed block; linear layers of
     block c >= 2 read the router output (anchors and block-1 layers read h_{l-1}).
+    With w_wg (L weights [H, D]; anchors' entries unused) the linear layers are
+    write-gated, the logits being W = u W_wg[l]^T.
 
     Returns y = h_L and, when keep_trace, a dict of per-layer lists
     u, Y, o (each [B, N, D]) and alpha ([B, N, c-1] or None), plus kinds."""
@@ -262,7 +288,8 @@ def stack(x, w_qkvg: Sequence[np.ndarray], w_o: Sequence[np.ndarray], w_r, H: in
         qkvg = project(u, w_qkvg[l - 1])
         q, k, v, g = (qkvg[..., i * D:(i + 1) * D] for i in range(4))
         if kind == "linear":
-            Y = linear_attn(q, k, v, g, H, eps)
+            wl = None if w_wg is None else project(u, w_wg[l - 1])
+            Y = linear_attn(q, k, v, g, H, eps, wgate=wl)
         else:
             Y = softmax_anchor(q, k, v, g, H)
         o = project(Y, w_o[l - 1])

@@ -48,6 +48,13 @@ def test_golden_gate(golden):
     np.testing.assert_allclose(O.gate(c["a"], c["g"]), c["expect"], rtol=0, atol=1e-14)
 
 
+def test_golden_write_gated_linear(golden):
+    c = golden["write_gated_linear_core"]
+    a = O.lin_core(np.array([c["q"]]), np.array([c["k"]]), np.array([c["v"]]), H=1,
+                   eps=c["eps"], wgate=np.array([c["wgate"]]))
+    np.testing.assert_allclose(a[0], c["expect"], rtol=0, atol=1e-14)
+
+
 def test_golden_route(golden):
     c = golden["route"]
     h = np.array([c["h"]])
@@ -121,6 +128,75 @@ def test_linear_state_rows_subset():
     rows = [0, 5, 32]
     np.testing.assert_allclose(O.lin_readout(q[:, rows], S, z, H, 1e-6),
                                O.lin_core(q, k, v, H)[:, rows], rtol=1e-14, atol=0)
+
+
+# ------------------------------------------------------------ write-gated linear core
+
+@pytest.mark.parametrize("N,H,d", [(1, 1, 4), (29, 2, 8), (64, 3, 16)])
+def test_write_gated_linear_equals_bruteforce(N, H, d):
+    q, k, v = (rand((2, N, H * d), s) for s in (70, 71, 72))
+    w = rand((2, N, H), 73, 3.0)
+    a = O.lin_core(q, k, v, H, eps=1e-6, wgate=w)
+    b = O.lin_core_bruteforce(q, k, v, H, eps=1e-6, wgate=w)
+    assert rel(a, b) < 1e-12
+    if N > 1:   # (one token: the gate cancels in the normalisation)
+        assert rel(a, O.lin_core(q, k, v, H, eps=1e-6)) > 1e-3
+
+
+def test_write_gate_open_is_ungated():
+    # sigmoid(40) = 1 - 4e-18: a wide-open write gate is the ungated layer
+    N, H, d = 45, 2, 8
+    q, k, v = (rand((1, N, H * d), s) for s in (74, 75, 76))
+    a = O.lin_core(q, k, v, H, wgate=np.full((1, N, H), 40.0))
+    assert rel(a, O.lin_core(q, k, v, H)) < 1e-15
+
+
+def test_write_gate_closed_token_is_removed():
+    # a token whose gate is shut (sigmoid(-80) ~ 2e-35) writes nothing into S
+    # or z: the result equals the layer run on the other tokens only, for the
+    # gated head; other heads still see the token
+    N, H, d = 20, 2, 8
+    q, k, v = (np.abs(rand((1, N, H * d), s)) for s in (77, 78, 79))
+    w = rand((1, N, H), 80)
+    w[0, 7, 1] = -80.0
+    a = O.lin_core(q, k, v, H, wgate=w)
+    keep = [t for t in range(N) if t != 7]
+    ref = O.lin_core(q, k[:, keep], v[:, keep], H, wgate=w[:, keep])
+    np.testing.assert_allclose(a[0, :, d:], ref[0, :, d:], rtol=1e-13, atol=0)
+    assert np.abs(a[0, :, :d] - ref[0, :, :d]).max() > 1e-3
+
+
+def test_write_gate_constant_cancels_up_to_eps():
+    # a constant gate omega scales S and z alike, so it only rescales eps:
+    # A = phi(Q) S / (phi(Q) z + eps / omega). This fails if only S is gated.
+    N, H, d, c, eps = 40, 2, 8, -1.5, 0.5
+    q, k, v = (rand((1, N, H * d), s) for s in (81, 82, 83))
+    om = 1.0 / (1.0 + math.exp(-c))
+    a = O.lin_core(q, k, v, H, eps=eps, wgate=np.full((1, N, H), c))
+    assert rel(a, O.lin_core(q, k, v, H, eps=eps / om)) < 1e-13
+    assert rel(a, O.lin_core(q, k, v, H, eps=eps)) > 1e-3
+
+
+def test_write_gate_heads_and_tokens_are_indexed_right():
+    # changing the logit of (token 3, head 1) changes head 1 only
+    N, H, d = 16, 3, 4
+    q, k, v = (np.abs(rand((1, N, H * d), s)) for s in (84, 85, 86))
+    w = rand((1, N, H), 87)
+    a = O.lin_core(q, k, v, H, wgate=w)
+    w2 = w.copy()
+    w2[0, 3, 1] += 2.0
+    a2 = O.lin_core(q, k, v, H, wgate=w2)
+    np.testing.assert_array_equal(a2[0, :, :d], a[0, :, :d])
+    np.testing.assert_array_equal(a2[0, :, 2 * d:], a[0, :, 2 * d:])
+    assert np.abs(a2[0, :, d:2 * d] - a[0, :, d:2 * d]).max() > 1e-4
+
+
+def test_write_weights_layout_and_values():
+    w = rand((2, 5, 3), 88, 4.0)
+    om = O.write_weights(w, 3)
+    assert om.shape == (2, 3, 5, 1)
+    from scipy.special import expit
+    np.testing.assert_allclose(om[1, 2, 4, 0], expit(w[1, 4, 2]), rtol=1e-15)
 
 
 # ------------------------------------------------------------ softmax core
@@ -303,6 +379,34 @@ def test_stack_single_block_attnres_on_equals_off():
     x, wq, wo, wr, H = small_stack(L=8)
     np.testing.assert_array_equal(O.stack(x, wq, wo, wr, H, attnres_block=8),
                                   O.stack(x, wq, wo, wr, H, attnres_block=0))
+
+
+def test_stack_zero_write_gate_weights_double_eps():
+    # W_wg = 0 gives every token the logit 0, a constant gate of 1/2, so the
+    # write-gated stack is the ungated one with eps doubled; anchors ignore
+    # their entry, so garbage there changes nothing
+    x, wq, wo, wr, H = small_stack(L=12)
+    D = x.shape[-1]
+    w0 = [np.zeros((H, D)) for _ in range(12)]
+    for l in (3, 7, 11):
+        w0[l] = rand((H, D), 90 + l)
+    y = O.stack(x, wq, wo, wr, H, eps=0.3, w_wg=w0)
+    np.testing.assert_allclose(y, O.stack(x, wq, wo, wr, H, eps=0.6), rtol=1e-12, atol=1e-13)
+    assert rel(y, O.stack(x, wq, wo, wr, H, eps=0.3)) > 1e-6
+
+
+def test_stack_write_gate_logits_come_from_the_layer_input():
+    # the logits of a routed linear layer are u W_wg^T with u the router output
+    x, wq, wo, wr, H = small_stack(L=12)
+    D = x.shape[-1]
+    wwg = [rand((H, D), 95 + l, 1 / math.sqrt(D)) for l in range(12)]
+    _, tr = O.stack(x, wq, wo, wr, H, w_wg=wwg, keep_trace=True)
+    l = 10                                   # layer 10 of block 2: routed, linear
+    u = tr["u"][l - 1]
+    qkvg = u @ wq[l - 1].T
+    q, k, v, g = (qkvg[..., i * D:(i + 1) * D] for i in range(4))
+    Y = O.gate(O.lin_core_bruteforce(q, k, v, H, wgate=u @ wwg[l - 1].T), g)
+    np.testing.assert_allclose(tr["Y"][l - 1], Y, rtol=1e-11, atol=1e-14)
 
 
 def test_stack_qkvg_column_order():

@@ -439,6 +439,55 @@ def run_case(args):
     return 0
 
 
+# 720p latent grid (23 x 40 patches) at 21 latent frames per 5 s of video; 60 s
+# at 16 fps gives 241 latent frames
+SWEEP_FRAMES = (21, 41, 81, 161, 241)
+
+
+def run_sweep(args):
+    """The hybrid's advantage over full softmax as the video gets longer: a
+    4-layer hybrid group (3 gated linear + 1 gated softmax) against 4 gated
+    softmax layers of the same width (D = 3072, H = 24), at 720p token counts
+    for 5 s to 60 s of video. One JSON line per length."""
+    import torch
+
+    import softmax_attention_video_gated_b200 as sva
+    import workloads as W
+
+    H, d, L = 24, 128, 4
+    D = H * d
+    std = 1.0 / math.sqrt(D)
+    wq = [W.normal_torch((4 * D, D), std, 99, W.TAG_WQKVG + l, "bf16") for l in range(1, L + 1)]
+    wo = [W.normal_torch((D, D), std, 99, W.TAG_WO + l, "bf16") for l in range(1, L + 1)]
+    for frames in SWEEP_FRAMES:
+        N = frames * 23 * 40
+        x = W.normal_torch((1, N, D), 1.0, 99, W.TAG_X, "bf16")
+        y = torch.empty_like(x)
+        res = {}
+        for name, all_sm in (("hybrid", False), ("all_softmax", True)):
+            st = sva.Stack(wq, wo, None, 1, N, H, attnres_block=0, all_softmax=all_sm)
+            ws = sva.workspace(st.workspace_bytes())
+            sva.sva_hybrid_stack_fwd(st, x, y, ws=ws)
+            torch.cuda.synchronize()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            for _ in range(args.steps):
+                sva.sva_hybrid_stack_fwd(st, x, y, ws=ws)
+            e1.record()
+            torch.cuda.synchronize()
+            if sva.sva_check_device_status(ws) != sva.SVA_OK:
+                raise RuntimeError("device status")
+            res[name] = e0.elapsed_time(e1) / args.steps
+            del ws
+        print(json.dumps({"sweep": "720p width, 4-layer group", "latent_frames": frames,
+                          "video_seconds_at_16fps": round((4 * (frames - 1) + 1) / 16, 1),
+                          "N": N, "hybrid_ms": res["hybrid"], "all_softmax_ms": res["all_softmax"],
+                          "speedup": res["all_softmax"] / res["hybrid"],
+                          "hybrid_tokens_per_s": N / (res["hybrid"] * 1e-3)}), flush=True)
+        del x, y
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
@@ -449,6 +498,8 @@ def main():
     ap.add_argument("--no-all-softmax", action="store_true")
     ap.add_argument("--case", choices=("anchor", "linear", "gemm", "proj_out"),
                     help="time one kernel class alone instead of the stack")
+    ap.add_argument("--sweep", action="store_true",
+                    help="hybrid vs all-softmax 4-layer groups at 5 s .. 60 s of 720p video")
     ap.add_argument("--B", type=int, default=1)
     ap.add_argument("--N", type=int, default=19320)
     ap.add_argument("--H", type=int, default=24)
@@ -458,6 +509,8 @@ def main():
     wl = dict(WORKLOAD)
     if args.case:
         return run_case(args)
+    if args.sweep:
+        return run_sweep(args)
     if args.impl == "reference":
         return run_reference(args, wl)
 

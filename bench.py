@@ -91,11 +91,14 @@ def algorithmic_work(kind: str, wl: dict, n_blocks_routed: int = 1):
     B, N, D = wl["B"], wl["N"], wl["H"] * wl["d"]
     M = B * N
     if kind == "proj_qkvg":
-        return "tensor", 2.0 * M * D * 4 * D
+        # write-gated stacks: the linear layers' projections also produce H logits
+        lin = 1.0 - 1.0 / wl["softmax_period"] if wl.get("write_gate") else 0.0
+        return "tensor", 2.0 * M * D * (4 * D + lin * wl["H"])
     if kind in ("proj_out", "keys"):
         return "tensor", 2.0 * M * D * D
     if kind == "linear_state":
-        return "hbm", 2.0 * M * D * 2
+        # (+ the write-gate logits, one bf16 per token and head, when gated)
+        return "hbm", 2.0 * M * D * 2 + (2.0 * M * wl["H"] if wl.get("write_gate") else 0.0)
     if kind == "linear_readout":
         return "hbm", 3.0 * M * D * 2
     if kind == "anchor":
@@ -227,8 +230,14 @@ def oracle_sample(wl: dict, frac: int):
     qkvg = O.project(x, wq)
     t["proj_qkvg"] = time.perf_counter() - t0
     q, k, v, g = (qkvg[..., i * D:(i + 1) * D] for i in range(4))
+    wgl = None
+    if wl.get("write_gate"):
+        wwg = W.normal((H, D), std, seed, W.TAG_WWG + 1, "bf16")
+        t0 = time.perf_counter()
+        wgl = O.project(x, wwg)
+        t["proj_wgate"] = time.perf_counter() - t0
     t0 = time.perf_counter()
-    y = O.linear_attn(q, k, v, g, H)
+    y = O.linear_attn(q, k, v, g, H, wgate=wgl)
     t["linear"] = time.perf_counter() - t0
     t0 = time.perf_counter()
     O.softmax_anchor(q, k, v, g, H)
@@ -249,7 +258,8 @@ def oracle_sample(wl: dict, frac: int):
     n_lin = L - n_anchor
     # routed linear layers: 6 in block 2 (one summary), 6 in block 3 (two)
     stack_s = (L * (t["proj_qkvg"] + t["proj_out"]) * r + n_lin * t["linear"] * r
-               + n_anchor * t["anchor"] * r * r + 6 * t["route1"] * r + 6 * t["route2"] * r)
+               + n_anchor * t["anchor"] * r * r + 6 * t["route1"] * r + 6 * t["route2"] * r
+               + n_lin * t.get("proj_wgate", 0.0) * r)
     desc = (f"fp64 oracle pieces at N_s = N/{frac} = {Ns} tokens, full D = {D}: one QKVG and one "
             f"output projection, one gated linear core, one gated softmax core, one 1-block and "
             f"one 2-block router; extrapolated to the 24-layer stack (x N/N_s, softmax core "
@@ -311,9 +321,18 @@ def make_stack(torch, sva, W, wl, all_softmax=False, weights=None):
         wo = [W.normal_torch((D, D), std, seed, W.TAG_WO + l, "bf16") for l in range(1, L + 1)]
         wr = W.normal_torch((D, D), std, seed, W.TAG_WR, "bf16")
         weights = (wq, wo, wr)
-    wq, wo, wr = weights
+    wq, wo, wr = weights[:3]
+    wwg = None
+    if wl.get("write_gate") and not all_softmax:
+        # write-gated linear layers: logits u W_wg^T, W_wg[l] [H, D]
+        if len(weights) < 4:
+            std = 1.0 / math.sqrt(D)
+            weights = weights + ([None if l % wl["softmax_period"] == 0 else
+                                  W.normal_torch((H, D), std, seed, W.TAG_WWG + l, "bf16")
+                                  for l in range(1, L + 1)],)
+        wwg = weights[3]
     st = sva.Stack(wq, wo, wr, B, N, H, softmax_period=wl["softmax_period"],
-                   attnres_block=wl["attnres_block"], all_softmax=all_softmax)
+                   attnres_block=wl["attnres_block"], all_softmax=all_softmax, w_wg=wwg)
     return st, weights
 
 
@@ -390,7 +409,7 @@ def run_case(args):
     B, N, H, d = args.B, args.N, args.H, 128
     D = H * d
     seed = 77
-    if args.case in ("anchor", "linear"):
+    if args.case in ("anchor", "linear", "linear_wg"):
         q, k, v, g = (W.normal_torch((B, N, D), 1.0, seed, tag, "bf16")
                       for tag in (W.TAG_Q, W.TAG_K, W.TAG_V, W.TAG_G))
         out = torch.empty_like(q)
@@ -400,8 +419,10 @@ def run_case(args):
             work, unit = 4.0 * B * N * N * D, "TFLOP/s"
         else:
             ws = sva.workspace(sva.sva_linear_attn_workspace_bytes(B, N, H, d, sva.SVA_BF16))
-            fn = lambda: sva.sva_linear_attn_fwd(q, k, v, g, out, H, ws=ws)  # noqa: E731
-            work, unit = 10.0 * B * N * D, "GB/s"
+            wg = (W.normal_torch((B, N, H), 1.0, seed, W.TAG_WGATE, "bf16")
+                  if args.case == "linear_wg" else None)
+            fn = lambda: sva.sva_linear_attn_fwd(q, k, v, g, out, H, ws=ws, wgate=wg)  # noqa: E731
+            work, unit = 10.0 * B * N * D + (2.0 * B * N * H if wg is not None else 0.0), "GB/s"
     elif args.case == "gemm":
         M, K, Nout = B * N, D, 4 * D
         x = W.normal_torch((M, K), 1.0, seed, W.TAG_X, "bf16")
@@ -496,10 +517,12 @@ def main():
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-all-softmax", action="store_true")
-    ap.add_argument("--case", choices=("anchor", "linear", "gemm", "proj_out"),
+    ap.add_argument("--case", choices=("anchor", "linear", "linear_wg", "gemm", "proj_out"),
                     help="time one kernel class alone instead of the stack")
     ap.add_argument("--sweep", action="store_true",
                     help="hybrid vs all-softmax 4-layer groups at 5 s .. 60 s of 720p video")
+    ap.add_argument("--write-gate", action="store_true",
+                    help="time the write-gated variant of the stack's linear layers")
     ap.add_argument("--B", type=int, default=1)
     ap.add_argument("--N", type=int, default=19320)
     ap.add_argument("--H", type=int, default=24)
@@ -507,6 +530,9 @@ def main():
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
     wl = dict(WORKLOAD)
+    if args.write_gate:
+        wl["name"] += ", write-gated linear layers"
+        wl["write_gate"] = True
     if args.case:
         return run_case(args)
     if args.sweep:

@@ -78,6 +78,9 @@ typedef struct {
   float eps;        /* linear attention: normaliser epsilon (e.g. 1e-6)       */
   float scale;      /* softmax anchor: logit scale; 0 means 1/sqrt(d)         */
   unsigned flags;   /* SVA_FLAG_*                                             */
+  const void* wgate; int64_t ldw;  /* linear attention, nullable [B, N, >=H]:
+                                      write-gate logits, one per token and head,
+                                      in dtype; row stride ldw >= H elements   */
 } sva_attn_args;
 
 /*
@@ -88,9 +91,14 @@ typedef struct {
  *     S = sum_t phi(K_t)^T V_t  (d x d),   z = sum_t phi(K_t)  (d)
  *     Y_t = phi(Q_t) S / (phi(Q_t) . z + eps)  *  sigmoid(G_t)   (per channel)
  *     out_t = Y_t (+ residual_t)
+ * Write-gated variant (wgate not NULL): the gate sets how much each token
+ * writes into the state [ai-papers.net summary, same section]; token t's term
+ * in both S and z is scaled by omega_t = sigmoid(wgate[b, t, h]):
+ *     S = sum_t omega_t phi(K_t)^T V_t,   z = sum_t omega_t phi(K_t).
  * Supported: SVA_BF16 with d = 128 (tcgen05 kernels), SVA_F32 with d in
  * {64, 128}. Any N >= 1. The workspace holds per-chunk partial states (fp32)
  * and the reduced state; size it with sva_linear_attn_workspace_bytes.
+ * The softmax anchor ignores wgate.
  */
 size_t sva_linear_attn_workspace_bytes(int B, int N, int H, int d, sva_dtype_t dtype);
 sva_status_t sva_linear_attn_fwd(const sva_attn_args* args, void* ws, size_t ws_bytes,
@@ -184,6 +192,10 @@ sva_status_t sva_attnres_route(const float* h, const void* const* keys,
  *       (AttnRes on), else h_{l-1}
  *   [Q | K | V | G] = u W_qkvg[l]^T;  Y = gated core;  h_l = h_{l-1} + Y W_o[l]^T
  * y = dtype(h_L). The residual stream h is kept in fp32 in the workspace.
+ * Write-gated linear layers: when w_wg is not NULL, linear layer l is the
+ * write-gated variant with logits u W_wg[l]^T (W_wg[l]: [H, D] in dtype;
+ * the entries of anchor layers are not read and may be NULL). The logits come
+ * out of the same GEMM as [Q | K | V | G].
  * Optional traces (any may be NULL): trace_o[l] receives o_l = Y W_o^T as
  * fp32 [B*N, D]; trace_y[l] receives Y as dtype [B*N, D]; trace_alpha[l]
  * receives the router weights fp32 [B*N, c-1] of routed layers.
@@ -221,6 +233,7 @@ typedef struct {
   int prof_capacity;
   int* prof_kind;              /* optional host array [prof_capacity]            */
   int* prof_count;             /* optional host int                              */
+  const void* const* w_wg;     /* optional, L pointers, each [H, D] in dtype     */
 } sva_stack_desc;
 
 size_t sva_hybrid_stack_workspace_bytes(const sva_stack_desc* desc);

@@ -48,6 +48,7 @@ class AttnArgs(ctypes.Structure):
         ("residual", ctypes.c_void_p), ("ldr", ctypes.c_int64),
         ("out", ctypes.c_void_p), ("ldo", ctypes.c_int64),
         ("eps", ctypes.c_float), ("scale", ctypes.c_float), ("flags", ctypes.c_uint),
+        ("wgate", ctypes.c_void_p), ("ldw", ctypes.c_int64),
     ]
 
 
@@ -62,6 +63,7 @@ class StackDesc(ctypes.Structure):
         ("trace_o", _c_void_p_p), ("trace_y", _c_void_p_p), ("trace_alpha", _c_void_p_p),
         ("prof_events", _c_void_p_p), ("prof_capacity", ctypes.c_int),
         ("prof_kind", ctypes.POINTER(ctypes.c_int)), ("prof_count", ctypes.POINTER(ctypes.c_int)),
+        ("w_wg", _c_void_p_p),
     ]
 
 
@@ -184,7 +186,7 @@ def workspace(nbytes: int, device=None):
                        device=device if device is not None else "cuda")
 
 
-def _attn_args(q, k, v, gate, out, H, residual, eps, scale, flags) -> AttnArgs:
+def _attn_args(q, k, v, gate, out, H, residual, eps, scale, flags, wgate=None) -> AttnArgs:
     B, N, D = q.shape
     if D % H:
         raise ValueError(f"width {D} is not a multiple of H={H}")
@@ -202,6 +204,13 @@ def _attn_args(q, k, v, gate, out, H, residual, eps, scale, flags) -> AttnArgs:
     if residual is not None:
         a.residual, a.ldr = _ptr(residual), _rows(residual, B, N)
     a.eps, a.scale, a.flags = float(eps), float(scale), int(flags)
+    if wgate is not None:
+        # [B, N, >=H] logits, one per token and head; rows ldw elements apart
+        if _dtype_code(wgate) != dt:
+            raise TypeError("wgate must have the dtype of q")
+        if wgate.dim() != 3 or wgate.shape[:2] != (B, N) or wgate.shape[2] < H:
+            raise ValueError(f"expected wgate [B={B}, N={N}, >={H}], got {tuple(wgate.shape)}")
+        a.wgate, a.ldw = _ptr(wgate), _rows(wgate, B, N)
     return a
 
 
@@ -214,9 +223,11 @@ def sva_linear_attn_workspace_bytes(B: int, N: int, H: int, d: int, dtype: int) 
 
 
 def sva_linear_attn_fwd(q, k, v, gate, out, H: int, residual=None, eps: float = 1e-6,
-                        flags: int = 0, ws=None, stream=None):
-    """Gated linear attention: out = phi(Q) S / (phi(Q).z + eps) * sigmoid(G) (+ residual)."""
-    a = _attn_args(q, k, v, gate, out, H, residual, eps, 0.0, flags)
+                        flags: int = 0, ws=None, stream=None, wgate=None):
+    """Gated linear attention: out = phi(Q) S / (phi(Q).z + eps) * sigmoid(G) (+ residual).
+    wgate [B, N, >=H] (optional): write-gate logits; token t's terms of S and z
+    are scaled by sigmoid(wgate[b, t, h])."""
+    a = _attn_args(q, k, v, gate, out, H, residual, eps, 0.0, flags, wgate)
     need = sva_linear_attn_workspace_bytes(a.B, a.N, a.H, a.d, a.dtype)
     ws = workspace(need, q.device) if ws is None else ws
     _check(_lib().sva_linear_attn_fwd(ctypes.byref(a), _ptr(ws), ws.numel(), _stream(stream)),
@@ -225,11 +236,11 @@ def sva_linear_attn_fwd(q, k, v, gate, out, H: int, residual=None, eps: float = 
 
 
 def sva_linear_attn_fwd_noalloc(q, k, v, gate, out, H: int, residual=None, eps: float = 1e-6,
-                                flags: int = 0, stream=None):
+                                flags: int = 0, stream=None, wgate=None):
     """sva_linear_attn_fwd without a workspace, for callers that cannot allocate
     device memory: the library's fixed 16 MiB device scratch is used instead.
     Calls that overlap on the GPU share that scratch and must be serialised."""
-    a = _attn_args(q, k, v, gate, out, H, residual, eps, 0.0, flags)
+    a = _attn_args(q, k, v, gate, out, H, residual, eps, 0.0, flags, wgate)
     _check(_lib().sva_linear_attn_fwd_noalloc(ctypes.byref(a), _stream(stream)),
            "sva_linear_attn_fwd_noalloc")
 
@@ -302,7 +313,7 @@ class Stack:
 
     def __init__(self, w_qkvg: Sequence, w_o: Sequence, w_r, B: int, N: int, H: int,
                  softmax_period: int = 4, attnres_block: int = 8, all_softmax: bool = False,
-                 eps: float = 1e-6, trace_o=None, trace_y=None, trace_alpha=None):
+                 eps: float = 1e-6, trace_o=None, trace_y=None, trace_alpha=None, w_wg=None):
         L = len(w_qkvg)
         D = w_qkvg[0].shape[1]
         d = StackDesc()
@@ -314,13 +325,14 @@ class Stack:
         d.w_o, a = _ptr_array(list(w_o)); self._keep.append(a)
         d.w_r = _ptr(w_r)
         d.eps = float(eps)
-        for name, ts in (("trace_o", trace_o), ("trace_y", trace_y), ("trace_alpha", trace_alpha)):
+        for name, ts in (("trace_o", trace_o), ("trace_y", trace_y), ("trace_alpha", trace_alpha),
+                         ("w_wg", w_wg)):
             p, a = _ptr_array(ts)
             if p is not None:
                 setattr(d, name, p)
                 self._keep.append(a)
         self.desc = d
-        self.tensors = (w_qkvg, w_o, w_r, trace_o, trace_y, trace_alpha)
+        self.tensors = (w_qkvg, w_o, w_r, trace_o, trace_y, trace_alpha, w_wg)
         self.prof_count = ctypes.c_int(0)
 
     def set_profile(self, events: Sequence, kinds_capacity: int):

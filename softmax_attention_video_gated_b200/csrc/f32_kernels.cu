@@ -31,7 +31,10 @@ __global__ void __launch_bounds__(256) gemm_f32_kernel(GemmArgs g) {
       const int r = idx / GK, c = idx % GK;
       const int64_t m = m0 + r, n = n0 + r, k = k0 + c;
       As[c][r] = (m < g.M && k < g.K) ? A[m * g.lda + k] : 0.f;
-      Bs[c][r] = (n < g.N && k < g.K) ? B[n * g.ldb + k] : 0.f;
+      const float* Bn = (g.b2 != nullptr && n >= g.n_split)
+                            ? static_cast<const float*>(g.b2) + (n - g.n_split) * g.ldb
+                            : B + n * g.ldb;
+      Bs[c][r] = (n < g.N && k < g.K) ? Bn[k] : 0.f;
     }
     __syncthreads();
 #pragma unroll
@@ -77,7 +80,8 @@ __global__ void __launch_bounds__(256) gemm_f32_kernel(GemmArgs g) {
 constexpr int LT = 32;  // tokens per smem tile
 
 // Partial state of one chunk of tokens of one (batch, head):
-// S_c = sum_t phi(K_t)^T V_t and z_c = sum_t phi(K_t).
+// S_c = sum_t phi(K_t)^T V_t and z_c = sum_t phi(K_t), each term times
+// sigmoid(wgate[b, t, h]) in the write-gated variant.
 template <int D_>
 __global__ void __launch_bounds__(256) lin_state_f32_kernel(sva_attn_args a, float* partial,
                                                             int tokens_per_chunk, int n_chunks) {
@@ -91,6 +95,7 @@ __global__ void __launch_bounds__(256) lin_state_f32_kernel(sva_attn_args a, flo
   const int t_begin = c * tokens_per_chunk;
   const int t_end = min(a.N, t_begin + tokens_per_chunk);
   const bool features = (a.flags & SVA_FLAG_QK_FEATURES) != 0;
+  const float* wg = static_cast<const float*>(a.wgate);
   float acc[R][R] = {};
   float zacc = 0.f;
   for (int t0 = t_begin; t0 < t_end; t0 += LT) {
@@ -103,6 +108,7 @@ __global__ void __launch_bounds__(256) lin_state_f32_kernel(sva_attn_args a, flo
         kv = K[row * a.ldk + h * D_ + col];
         vv = V[row * a.ldv + h * D_ + col];
         if (!features) kv = relu_f(kv);
+        if (wg != nullptr) kv *= 1.0f / (1.0f + expf(-wg[row * a.ldw + h]));  // write gate
       }
       Ks[r][col] = kv;
       Vs[r][col] = vv;

@@ -20,7 +20,10 @@
 //               update h += C (fp32) with an optional bf16 copy of h. Each warp
 //               releases the accumulator on rank 0's barrier.
 // Tiles run in groups of whole M-tile columns so one wave touches few A rows
-// and few B rows and both stay in L2.
+// and few B rows and both stay in L2. A ragged last N tile issues MMAs only as
+// wide as its columns (rounded up to 32), and the output columns from n_split
+// on may come from a second weight (the write-gate projection appended to the
+// fused [Q | K | V | G] projection, so the layer input is read once).
 #include <algorithm>
 
 #include "common.cuh"
@@ -72,6 +75,14 @@ __device__ __forceinline__ bool drain_wait(uint64_t* bar, uint32_t parity) {
   return mbar_wait(bar, parity, &never, nullptr, 0);
 }
 
+// MMA width of an N tile: the full BN, or for the ragged last tile its width
+// rounded up to 32 (a legal N for M = 256 on a CTA pair), so a narrow tail
+// costs tensor-core time in proportion to its width
+__device__ __forceinline__ int tile_n_mma(int64_t N, int64_t n0) {
+  const int64_t rem = N - n0;
+  return rem >= BN ? BN : static_cast<int>((rem + 31) / 32 * 32);
+}
+
 __device__ __forceinline__ void tile_coords(int tile, int m_tiles, int n_tiles, int group,
                                             int& m_blk, int& n_blk) {
   const int per_group = group * n_tiles;
@@ -86,6 +97,7 @@ template <int EPI>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     gemm_bf16_tc_kernel(const __grid_constant__ CUtensorMap map_a,
                         const __grid_constant__ CUtensorMap map_b,
+                        const __grid_constant__ CUtensorMap map_b2,
                         const __grid_constant__ CUtensorMap map_h,
                         const __grid_constant__ CUtensorMap map_c, GemmArgs g, int group) {
   constexpr int STAGES = Layout<EPI>::STAGES;
@@ -126,6 +138,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   if (warp == 0 && lane == 0) {
     tma_prefetch_desc(&map_a);
     tma_prefetch_desc(&map_b);
+    if (g.b2 != nullptr) tma_prefetch_desc(&map_b2);
     if (EPI == EPI_RESIDUAL) {
       tma_prefetch_desc(&map_h);
       tma_prefetch_desc(&map_c);
@@ -147,6 +160,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       for (int tile = cluster; tile < num_tiles && ok; tile += n_clusters) {
         int m_blk, n_blk;
         tile_coords(tile, m_tiles, n_tiles, group, m_blk, n_blk);
+        // each CTA of the pair holds half of the tile's MMA width of B rows
+        const int64_t n0 = static_cast<int64_t>(n_blk) * BN;
+        const bool second = g.b2 != nullptr && n0 >= g.n_split;
+        const CUtensorMap* mb = second ? &map_b2 : &map_b;
+        const int b_row = static_cast<int>(second ? n0 - g.n_split : n0) +
+                          static_cast<int>(rank) * (tile_n_mma(g.N, n0) / 2);
         for (int kb = 0; kb < k_blocks; ++kb) {
           if (!mbar_wait(&tl->empty[stage], phase ^ 1, abort_flag, g.status, WHERE_GEMM)) {
             ok = false;
@@ -155,7 +174,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           const uint32_t full0 = cluster_map(&tl->full[stage], 0);
           if (rank == 0) mbar_arrive_expect_tx(&tl->full[stage], 2 * STAGE_BYTES);
           tma_load_2d_pair(&map_a, full0, sA + stage * A_STAGE, kb * BK, m_blk * BM + rank * HALF);
-          tma_load_2d_pair(&map_b, full0, sB + stage * B_STAGE, kb * BK, n_blk * BN + rank * HALF);
+          tma_load_2d_pair(mb, full0, sB + stage * B_STAGE, kb * BK, b_row);
           ++issued;
           if (++stage == STAGES) {
             stage = 0;
@@ -172,12 +191,15 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   } else if (warp == 1) {
     if (lane == 0 && rank == 0) {
       // ------------------------------------------------ MMA issuer (rank 0 only)
-      constexpr uint32_t idesc = idesc_bf16_f32(BM, BN, false, false);
       int stage = 0;
       uint32_t phase = 0;
       int local = 0;
       bool ok = true;
       for (int tile = cluster; tile < num_tiles && ok; tile += n_clusters, ++local) {
+        int m_blk, n_blk;
+        tile_coords(tile, m_tiles, n_tiles, group, m_blk, n_blk);
+        const uint32_t idesc =
+            idesc_bf16_f32(BM, tile_n_mma(g.N, static_cast<int64_t>(n_blk) * BN), false, false);
         const int acc = local & 1;
         const uint32_t acc_phase = (local >> 1) & 1;
         if (!mbar_wait(&tl->acc_empty[acc], acc_phase ^ 1, abort_flag, g.status, WHERE_GEMM)) {
@@ -385,8 +407,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 }
 
 template <int EPI>
-cudaError_t launch(const CUtensorMap& ma, const CUtensorMap& mb, const CUtensorMap& mh,
-                   const CUtensorMap& mc, const GemmArgs& g, int grid, int group, cudaStream_t s) {
+cudaError_t launch(const CUtensorMap& ma, const CUtensorMap& mb, const CUtensorMap& mb2,
+                   const CUtensorMap& mh, const CUtensorMap& mc, const GemmArgs& g, int grid,
+                   int group, cudaStream_t s) {
   auto kern = gemm_bf16_tc_kernel<EPI>;
   constexpr size_t kGemmSmem = gemm_smem<EPI>();
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -404,13 +427,13 @@ cudaError_t launch(const CUtensorMap& ma, const CUtensorMap& mb, const CUtensorM
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, kern, ma, mb, mh, mc, g, group);
+  return cudaLaunchKernelEx(&cfg, kern, ma, mb, mb2, mh, mc, g, group);
 }
 
 }  // namespace
 
 cudaError_t gemm_bf16(const GemmArgs& g, cudaStream_t s) {
-  CUtensorMap ma, mb;
+  CUtensorMap ma, mb, mb2;
   {
     const uint64_t dims[2] = {static_cast<uint64_t>(g.K), static_cast<uint64_t>(g.M)};
     const uint64_t strides[1] = {static_cast<uint64_t>(g.lda) * 2};
@@ -419,11 +442,23 @@ cudaError_t gemm_bf16(const GemmArgs& g, cudaStream_t s) {
                      CU_TENSOR_MAP_SWIZZLE_128B))
       return cudaErrorInvalidValue;
   }
+  if (g.b2 != nullptr && (g.n_split <= 0 || g.n_split % BN != 0 || g.n_split >= g.N))
+    return cudaErrorInvalidValue;
+  const int64_t n_first = g.b2 != nullptr ? g.n_split : g.N;  // rows of b
   {
-    const uint64_t dims[2] = {static_cast<uint64_t>(g.K), static_cast<uint64_t>(g.N)};
+    const uint64_t dims[2] = {static_cast<uint64_t>(g.K), static_cast<uint64_t>(n_first)};
     const uint64_t strides[1] = {static_cast<uint64_t>(g.ldb) * 2};
     const uint32_t box[2] = {BK, HALF};
     if (!encode_tmap(&mb, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, g.b, dims, strides, box,
+                     CU_TENSOR_MAP_SWIZZLE_128B))
+      return cudaErrorInvalidValue;
+  }
+  mb2 = mb;
+  if (g.b2 != nullptr) {
+    const uint64_t dims[2] = {static_cast<uint64_t>(g.K), static_cast<uint64_t>(g.N - g.n_split)};
+    const uint64_t strides[1] = {static_cast<uint64_t>(g.ldb) * 2};
+    const uint32_t box[2] = {BK, HALF};
+    if (!encode_tmap(&mb2, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, g.b2, dims, strides, box,
                      CU_TENSOR_MAP_SWIZZLE_128B))
       return cudaErrorInvalidValue;
   }
@@ -434,7 +469,7 @@ cudaError_t gemm_bf16(const GemmArgs& g, cudaStream_t s) {
   // a wave of clusters covers `group` M tiles by about four N tiles
   const int group = static_cast<int>(std::max<int64_t>(
       1, std::min<int64_t>(m_tiles, clusters / std::min<int64_t>(4, n_tiles))));
-  if (g.epi == EPI_STORE) return launch<EPI_STORE>(ma, mb, ma, ma, g, 2 * clusters, group, s);
+  if (g.epi == EPI_STORE) return launch<EPI_STORE>(ma, mb, mb2, ma, ma, g, 2 * clusters, group, s);
   // residual epilogue: h (fp32, 32x32 boxes, 128-byte swizzle) and its bf16
   // copy (32x32 boxes, 64-byte swizzle); without a copy the h map stands in
   CUtensorMap mh, mc;
@@ -455,7 +490,7 @@ cudaError_t gemm_bf16(const GemmArgs& g, cudaStream_t s) {
                      CU_TENSOR_MAP_SWIZZLE_64B))
       return cudaErrorInvalidValue;
   }
-  return launch<EPI_RESIDUAL>(ma, mb, mh, mc, g, 2 * clusters, group, s);
+  return launch<EPI_RESIDUAL>(ma, mb, mb2, mh, mc, g, 2 * clusters, group, s);
 }
 
 }  // namespace sva

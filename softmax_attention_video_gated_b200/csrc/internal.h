@@ -55,6 +55,10 @@ enum GemmEpi { EPI_STORE = 0, EPI_RESIDUAL = 1 };
 struct GemmArgs {
   const void* a = nullptr;  int64_t lda = 0;   // [M, K]
   const void* b = nullptr;  int64_t ldb = 0;   // [N, K]
+  // optional second weight: output columns n >= n_split take row n - n_split
+  // of b2 ([N - n_split, K], row stride ldb) instead of row n of b; n_split is
+  // a multiple of 256 (the tile width of the tensor-core path)
+  const void* b2 = nullptr; int64_t n_split = 0;
   int64_t M = 0, N = 0, K = 0;
   int epi = EPI_STORE;
   void* c = nullptr;        int64_t ldc = 0;   // EPI_STORE: [M, N] output

@@ -4,6 +4,9 @@
 // [ai-papers.net summary, section "ハイブリッド線形アテンション"]. With phi = ReLU:
 //   S = sum_t phi(K_t)^T V_t,  z = sum_t phi(K_t),
 //   Y_t = phi(Q_t) S / (phi(Q_t) . z + eps) * sigmoid(G_t)   (+ residual).
+// In the write-gated variant token t's terms of S and z carry the factor
+// sigmoid(W_t), one logit per token and head (same section: the gate sets how
+// much each token writes into the state).
 //
 // Three kernels, all HBM-bound (the roofline is 10 B*N*D bytes of Q, K, V, G
 // and Y traffic per layer):
@@ -55,10 +58,15 @@ __device__ __forceinline__ bool drain_wait(uint64_t* bar, uint32_t parity) {
   return mbar_wait(bar, parity, &never, nullptr, 0);
 }
 
+// kWriteGate: token t's row of phi(K) is scaled by omega_t = sigmoid(wgate[b, t, h])
+// before it enters S and z (the write-gated variant); wgate is [B, N, >=H], row
+// stride ldw.
+template <bool kWriteGate>
 __global__ void __launch_bounds__(192, 1)
     lin_state_tc_kernel(const __grid_constant__ CUtensorMap map_k,
                         const __grid_constant__ CUtensorMap map_v, int N, int H,
-                        int tiles_per_chunk, int n_chunks, unsigned flags, float* partial,
+                        int tiles_per_chunk, int n_chunks, unsigned flags,
+                        const __nv_bfloat16* __restrict__ wgate, int64_t ldw, float* partial,
                         int* status) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -169,7 +177,25 @@ __global__ void __launch_bounds__(192, 1)
     int stage = 0;
     uint32_t phase = 0;
     bool ok = true;
+    // Write gate: a warp's threads touch 32 rows of a tile (row classes rc,
+    // rc + 1 and every 8th row after them); lane L fetches the logit of the
+    // row (rc & ~1) + (L & 1) + 8 (L >> 1) one tile ahead and the others read
+    // its sigmoid by shuffle, so each tile costs one load per lane.
+    const int my_row = (rc & ~1) + (lane & 1) + 8 * (lane >> 1);
+    auto load_logit = [&](int tile) -> float {
+      const int t = tile * TT + my_row;
+      return t < N ? __bfloat162float(wgate[(static_cast<int64_t>(b) * N + t) * ldw + h]) : 0.f;
+    };
+    float next_logit = 0.f;
+    if constexpr (kWriteGate) {
+      if (ntiles > 0) next_logit = load_logit(tile0);
+    }
     for (int i = 0; i < ntiles; ++i) {
+      float om_lane = 1.f;
+      if constexpr (kWriteGate) {
+        om_lane = 1.0f / (1.0f + __expf(-next_logit));
+        if (i + 1 < ntiles) next_logit = load_logit(tile0 + i + 1);
+      }
       bool w = mbar_wait(&tl->full[stage], phase, abort_flag, status, WHERE_LIN_STATE);
       if (!__all_sync(0xffffffffu, w)) {
         ok = false;
@@ -180,7 +206,19 @@ __global__ void __launch_bounds__(192, 1)
       for (int j = 0; j < TT / 8; ++j) {
         uint4* p = reinterpret_cast<uint4*>(kt + (rc + 8 * j) * 128);
         uint4 v = *p;
-        if (!features) {
+        if constexpr (kWriteGate) {
+          // phi(K) * omega, rounded once to bf16: S and z see the same values
+          const float o = __shfl_sync(0xffffffffu, om_lane, (rc & 1) + 2 * j);
+          const uint32_t in[4] = {v.x, v.y, v.z, v.w};
+          uint32_t r4[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const uint32_t f = features ? in[e] : relu_bf16x2(in[e]);
+            r4[e] = pack_bf16x2(bf16lo_to_f32(f) * o, bf16hi_to_f32(f) * o);
+          }
+          v = make_uint4(r4[0], r4[1], r4[2], r4[3]);
+          *p = v;
+        } else if (!features) {
           v.x = relu_bf16x2(v.x);
           v.y = relu_bf16x2(v.y);
           v.z = relu_bf16x2(v.z);
@@ -531,12 +569,15 @@ cudaError_t linear_bf16(const sva_attn_args& a, int* status, void* scratch, cuda
   cudaError_t e;
   {
     ProfScope ps(prof, s, SVA_KERNEL_LINEAR_STATE);
-    e = cudaFuncSetAttribute(lin_state_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    const bool wg = a.wgate != nullptr;
+    auto kern = wg ? lin_state_tc_kernel<true> : lin_state_tc_kernel<false>;
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(kStateSmem));
     if (e != cudaSuccess) return e;
     dim3 grid(p.n_chunks, a.H, a.B);
-    lin_state_tc_kernel<<<grid, 192, kStateSmem, s>>>(mk, mv, a.N, a.H, p.tiles_per_chunk,
-                                                      p.n_chunks, a.flags, partial, status);
+    kern<<<grid, 192, kStateSmem, s>>>(mk, mv, a.N, a.H, p.tiles_per_chunk, p.n_chunks, a.flags,
+                                       static_cast<const __nv_bfloat16*>(a.wgate), a.ldw,
+                                       partial, status);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
   {

@@ -77,6 +77,9 @@ extern "C" sva_status_t sva_linear_attn_fwd_noalloc(const sva_attn_args* a, sva_
   if (a->residual != nullptr && (!ptr_ok(a->residual) || !row_ok(a->ldr, D, es)))
     return SVA_ERR_INVALID_ARGUMENT;
   if (!(a->eps >= 0.f && std::isfinite(a->eps))) return SVA_ERR_INVALID_ARGUMENT;
+  if (a->wgate != nullptr &&
+      (a->ldw < a->H || reinterpret_cast<uintptr_t>(a->wgate) % es != 0))
+    return SVA_ERR_INVALID_ARGUMENT;
   if (static_cast<int64_t>(a->B) * a->N > (int64_t(1) << 31)) return SVA_ERR_UNSUPPORTED;
   if (a->dtype == SVA_BF16 && a->d != 128) return SVA_ERR_UNSUPPORTED;
   if (a->dtype == SVA_F32 && a->d != 64 && a->d != 128) return SVA_ERR_UNSUPPORTED;

@@ -108,6 +108,9 @@ sva_status_t check_attn(const sva_attn_args* a, bool linear) {
     if (!aligned16(ptrs[i]) || !ld_ok(lds[i], D, a->dtype)) return SVA_ERR_INVALID_ARGUMENT;
   }
   if (linear && !(a->eps >= 0.f && std::isfinite(a->eps))) return SVA_ERR_INVALID_ARGUMENT;
+  if (linear && a->wgate != nullptr &&
+      (a->ldw < a->H || reinterpret_cast<uintptr_t>(a->wgate) % esize(a->dtype) != 0))
+    return SVA_ERR_INVALID_ARGUMENT;
   if (!linear && !(std::isfinite(a->scale) && a->scale >= 0.f)) return SVA_ERR_INVALID_ARGUMENT;
   if (static_cast<int64_t>(a->B) * a->N > (int64_t(1) << 31)) return SVA_ERR_UNSUPPORTED;
   if (a->dtype == SVA_BF16 && a->d != 128) return SVA_ERR_UNSUPPORTED;
@@ -311,6 +314,14 @@ int summaries_needed(const sva_stack_desc& d) {
   return need;
 }
 
+// Row stride of the fused projection output [Q | K | V | G (| W)]: 4D, plus,
+// for write-gated stacks, the H write-gate logits padded to 8 elements so
+// rows stay 16-byte aligned for the TMA maps that read Q, K, V and G.
+int64_t qkvg_ld(const sva_stack_desc& d) {
+  const int64_t D = static_cast<int64_t>(d.H) * d.d;
+  return 4 * D + (d.w_wg != nullptr ? (static_cast<int64_t>(d.H) + 7) / 8 * 8 : 0);
+}
+
 StackLayout stack_layout(const sva_stack_desc& d) {
   StackLayout s{};
   const size_t rows = static_cast<size_t>(d.B) * d.N;
@@ -325,7 +336,7 @@ StackLayout stack_layout(const sva_stack_desc& d) {
   };
   s.h = take(rows * D * 4);
   s.u = take(rows * D * es);
-  s.qkvg = take(rows * 4 * D * es);
+  s.qkvg = take(rows * static_cast<size_t>(qkvg_ld(d)) * es);
   s.y = take(rows * D * es);
   s.lin = take(linear_plan(d.B, d.N, d.H, d.d, d.dtype).total);
   s.n_summ = summaries_needed(d);
@@ -353,6 +364,10 @@ sva_status_t check_stack(const sva_stack_desc* d) {
   if (n_summ > 8) return SVA_ERR_UNSUPPORTED;
   if (n_summ > 0 && (d->w_r == nullptr || !aligned16(d->w_r))) return SVA_ERR_INVALID_ARGUMENT;
   if (d->prof_events != nullptr && d->prof_capacity < 0) return SVA_ERR_INVALID_ARGUMENT;
+  if (d->w_wg != nullptr)
+    for (int l = 1; l <= d->L; ++l)
+      if (!layer_is_anchor(*d, l) && (d->w_wg[l - 1] == nullptr || !aligned16(d->w_wg[l - 1])))
+        return SVA_ERR_INVALID_ARGUMENT;
   return SVA_OK;
 }
 
@@ -397,6 +412,7 @@ extern "C" sva_status_t sva_hybrid_stack_fwd(const sva_stack_desc* desc, const v
   auto summ = [&](int c) { return base + lay.summ + static_cast<size_t>(c - 1) * act_bytes; };
   auto keyb = [&](int c) { return base + lay.keys + static_cast<size_t>(c - 1) * act_bytes; };
   const bool bf16 = d.dtype == SVA_BF16;
+  const int64_t ldp = qkvg_ld(d);
 
   cudaError_t e = cudaSuccess;
 #define SVA_TRY(expr)                          \
@@ -432,12 +448,20 @@ extern "C" sva_status_t sva_hybrid_stack_fwd(const sva_stack_desc* desc, const v
       SVA_TRY(route(h, ks, ss, c - 1, u, alpha, rows, D, d.dtype, s));
       in = u;
     }
+    const bool write_gated = !anchor && d.w_wg != nullptr;
     {
-      // [Q | K | V | G] = u W_qkvg^T; the linear layers take phi(Q), phi(K) from the epilogue
+      // [Q | K | V | G] = u W_qkvg^T; the linear layers take phi(Q), phi(K) from
+      // the epilogue; a write-gated layer's logits u W_wg^T follow in the same
+      // GEMM as columns 4D .. 4D + H
       GemmArgs g;
       g.a = in; g.lda = D; g.b = d.w_qkvg[l - 1]; g.ldb = D;
       g.M = rows; g.N = 4 * static_cast<int64_t>(D); g.K = D;
-      g.epi = EPI_STORE; g.c = qkvg; g.ldc = 4 * static_cast<int64_t>(D);
+      if (write_gated) {
+        g.b2 = d.w_wg[l - 1];
+        g.n_split = g.N;
+        g.N += d.H;
+      }
+      g.epi = EPI_STORE; g.c = qkvg; g.ldc = ldp;
       g.relu_cols = anchor ? 0 : 2 * D;
       g.status = status;
       ProfScope ps(prof, s, SVA_KERNEL_PROJ_QKVG);
@@ -446,11 +470,15 @@ extern "C" sva_status_t sva_hybrid_stack_fwd(const sva_stack_desc* desc, const v
     sva_attn_args a{};
     a.B = d.B; a.N = d.N; a.H = d.H; a.d = d.d; a.dtype = d.dtype;
     a.q = qkvg; a.k = qkvg + D * es; a.v = qkvg + 2 * D * es; a.gate = qkvg + 3 * D * es;
-    a.ldq = a.ldk = a.ldv = a.ldg = 4 * static_cast<int64_t>(D);
+    a.ldq = a.ldk = a.ldv = a.ldg = ldp;
     a.residual = nullptr; a.ldr = 0;
     a.out = ybuf; a.ldo = D;
     a.eps = d.eps; a.scale = 0.f;
     a.flags = anchor ? 0u : SVA_FLAG_QK_FEATURES;
+    if (write_gated) {
+      a.wgate = qkvg + 4 * D * es;
+      a.ldw = ldp;
+    }
     if (anchor) {
       ProfScope ps(prof, s, SVA_KERNEL_ANCHOR);
       SVA_TRY(bf16 ? anchor_bf16(a, status, s) : anchor_f32(a, status, s));

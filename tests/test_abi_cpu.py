@@ -55,11 +55,15 @@ def _args(**kw):
     (dict(d=64, ldq=128, ldk=128, ldv=128, ldg=128, ldo=128), sva.SVA_ERR_UNSUPPORTED),
     (dict(eps=-1.0), sva.SVA_ERR_INVALID_ARGUMENT),
     (dict(dtype=7), sva.SVA_ERR_INVALID_ARGUMENT),
+    (dict(wgate=0x30000, ldw=1), sva.SVA_ERR_INVALID_ARGUMENT),  # write gate: ldw < H
+    (dict(wgate=0x30001, ldw=8), sva.SVA_ERR_INVALID_ARGUMENT),  # not element-aligned
 ])
 def test_linear_attn_rejects_bad_arguments_on_host(bad, expect):
     a = _args(**bad)
     st = sva._lib().sva_linear_attn_fwd(ctypes.byref(a), 0x20000, 1 << 30, None)
     assert st == expect
+    # the allocation-free entry point validates the same way
+    assert sva._lib().sva_linear_attn_fwd_noalloc(ctypes.byref(a), None) == expect
 
 
 def test_workspace_checks_happen_before_launch():
@@ -106,4 +110,13 @@ def test_stack_workspace_query_and_validation():
     assert lib.sva_hybrid_stack_fwd(ctypes.byref(d), 0x10000, 0x20000, 0x30000, 1 << 40,
                                     None) == sva.SVA_ERR_INVALID_ARGUMENT
     d.attnres_block = 0  # AttnRes off: no router projection needed
-    assert lib.sva_hybrid_stack_workspace_bytes(ctypes.byref(d)) > 0
+    n0 = lib.sva_hybrid_stack_workspace_bytes(ctypes.byref(d))
+    assert n0 > 0
+    # write-gated linear layers: the fused projection output gains 24 columns; anchors' entries
+    # may be NULL, linear layers' may not
+    wg = (ctypes.c_void_p * L)(*[None if l % 4 == 3 else 0x300000 for l in range(L)])
+    d.w_wg = ctypes.cast(wg, ctypes.POINTER(ctypes.c_void_p))
+    n1 = lib.sva_hybrid_stack_workspace_bytes(ctypes.byref(d))
+    assert rows * 24 * 2 <= n1 - n0 <= rows * 24 * 2 + 2048
+    wg[0] = None
+    assert lib.sva_hybrid_stack_workspace_bytes(ctypes.byref(d)) == 0

@@ -69,6 +69,22 @@ def test_720p_layer_sampled_rows(core720, kind):
     check_rows(kind, x, out, W.STACK720P.H, sample_rows(W.STACK720P.N))
 
 
+def test_720p_write_gated_linear_layer_sampled_rows(core720):
+    # write-gate logits [B, N, H] ~ N(0, 1), the spread of u W_wg^T at the
+    # stack's weight scale
+    x, t = core720
+    w = W.STACK720P
+    wg = W.normal((w.B, w.N, w.H), 1.0, w.seed, W.TAG_WGATE, "bf16")
+    out = torch.empty_like(t["q"])
+    ws = sva.sva_linear_attn_fwd(t["q"], t["k"], t["v"], t["g"], out, w.H, eps=1e-6,
+                                 wgate=to_dev(wg, "bf16"))
+    assert sva.sva_check_device_status(ws) == sva.SVA_OK
+    rows = sample_rows(w.N, seed=2)
+    ref = O.linear_attn(x["q"][:, rows], x["k"], x["v"], x["g"][:, rows], w.H, eps=1e-6, wgate=wg)
+    assert_close(to_host(out[:, torch.as_tensor(rows, device="cuda")]), ref, "bf16",
+                 "720p write-gated linear sampled rows")
+
+
 # ------------------------------------------------------------------ long video (N = 37,720)
 
 def test_long_video_layers_sampled_rows():

@@ -140,6 +140,59 @@ def test_linear_attn_zero_query_rows_are_zero_not_nan():
     assert np.all(o[0, 17] == 0.0)
 
 
+# ------------------------------------------------------------------ write-gated linear attention
+
+def wgate_case(B, N, H, dtype, seed, width, std=2.0):
+    """Write-gate logits [B, N, H] ~ N(0, std^2), handed to the library as the
+    first H columns of a [B, N, width] buffer (row stride width)."""
+    w = W.normal((B, N, width), std, seed, W.TAG_WGATE, dtype)
+    return w[..., :H], to_dev(w, dtype)[..., :H]
+
+
+@pytest.mark.parametrize("dtype,d", [("bf16", 128), ("f32", 64), ("f32", 128)])
+@pytest.mark.parametrize("B,N,H,width", [(1, 1, 1, 8), (2, 1000, 2, 2), (1, 3001, 3, 8), (2, 129, 2, 5)])
+def test_write_gated_linear_attn(dtype, d, B, N, H, width):
+    x, t = core_case(B, N, H, d, dtype, seed=41 + N)
+    wg, twg = wgate_case(B, N, H, dtype, 42 + N, width)
+    out = torch.empty_like(t["q"])
+    ws = sva.sva_linear_attn_fwd(t["q"], t["k"], t["v"], t["g"], out, H, eps=1e-6, wgate=twg)
+    assert sva.sva_check_device_status(ws) == sva.SVA_OK
+    ref = O.linear_attn(x["q"], x["k"], x["v"], x["g"], H, eps=1e-6, wgate=wg)
+    assert_close(to_host(out), ref, dtype, f"write-gated linear B={B} N={N}")
+    if N > 1:   # the gate changes the result by far more than the tolerance
+        assert rel_l2(ref, O.linear_attn(x["q"], x["k"], x["v"], x["g"], H, eps=1e-6)) > 0.05
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_write_gated_linear_attn_saturated_gates_and_features(dtype):
+    # logits ~ N(0, 30^2): most gates are shut or wide open; q and k given as
+    # features (flag) in a fused buffer, as the stack calls it
+    B, N, H, d = 1, 1500, 2, 128
+    D = H * d
+    x, _ = core_case(B, N, H, d, dtype, seed=43)
+    wg, twg = wgate_case(B, N, H, dtype, 44, 8, std=30.0)
+    fq, fk = O.phi(x["q"]).astype(np.float32), O.phi(x["k"]).astype(np.float32)
+    buf = to_dev(np.concatenate([fq, fk, x["v"], x["g"]], axis=-1), dtype)
+    out = torch.empty(B, N, D, device="cuda", dtype=TDT[dtype])
+    ws = sva.sva_linear_attn_fwd(buf[..., :D], buf[..., D:2 * D], buf[..., 2 * D:3 * D],
+                                 buf[..., 3 * D:], out, H, eps=1e-6,
+                                 flags=sva.SVA_FLAG_QK_FEATURES, wgate=twg)
+    assert sva.sva_check_device_status(ws) == sva.SVA_OK
+    ref = O.linear_attn(x["q"], x["k"], x["v"], x["g"], H, eps=1e-6, wgate=wg)
+    assert_close(to_host(out), ref, dtype, "write-gated linear, saturated gates")
+
+
+def test_write_gated_linear_attn_noalloc_matches_workspace_call():
+    B, N, H, d = 2, 700, 2, 128
+    x, t = core_case(B, N, H, d, "bf16", seed=45)
+    _, twg = wgate_case(B, N, H, "bf16", 46, 4)
+    out1, out2 = torch.empty_like(t["q"]), torch.empty_like(t["q"])
+    sva.sva_linear_attn_fwd(t["q"], t["k"], t["v"], t["g"], out1, H, wgate=twg)
+    sva.sva_linear_attn_fwd_noalloc(t["q"], t["k"], t["v"], t["g"], out2, H, wgate=twg)
+    torch.cuda.synchronize()
+    assert torch.equal(out1, out2)
+
+
 # ------------------------------------------------------------------ gated softmax anchor
 
 @pytest.mark.parametrize("dtype,d", [("bf16", 128), ("f32", 64), ("f32", 128)])
@@ -284,6 +337,52 @@ def test_stack_bf16_three_blocks_with_router():
             assert_close(alpha_rows(tra[l], x.shape[1], nb), tr["alpha"][l][0], "bf16",
                          f"alpha_{l + 1}")
     assert_close(y - x, yref - x, "bf16", "y - x")
+
+
+def wwg_weights(L, H, D, dtype, seed):
+    return [W.normal((H, D), 1.0 / math.sqrt(D), seed, W.TAG_WWG + l, dtype) for l in range(1, L + 1)]
+
+
+def run_wg_stack(x, wq, wo, wr, wwg, H, dtype, **kw):
+    return run_stack(x, wq, wo, wr, H, dtype,
+                     w_wg=[None if l % 4 == 0 else to_dev(w, dtype)
+                           for l, w in enumerate(wwg, start=1)], **kw)
+
+
+def test_stack_bf16_write_gated_two_blocks():
+    x, wq, wo, wr, H = small_bf16_stack(12, N=333, seed=93)
+    wwg = wwg_weights(12, H, x.shape[-1], "bf16", 93)
+    y, tro, tra = run_wg_stack(x, wq, wo, wr, wwg, H, "bf16")
+    yref, tr = O.stack(x, wq, wo, wr, H, keep_trace=True, w_wg=wwg)
+    for l in range(12):
+        assert_close(tro[l], tr["o"][l], "bf16", f"o_{l + 1}")
+    assert_close(y - x, yref - x, "bf16", "y - x")
+    assert rel_l2(yref - x, O.stack(x, wq, wo, wr, H) - x) > 0.05   # the gate matters
+
+
+def test_stack_fp32_write_gated_hybrid_group():
+    w = W.HYBRID4_F32
+    x = W.stack_x(w)
+    p = W.stack_weights(w)
+    wwg = wwg_weights(w.L, w.H, w.D, "f32", w.seed)
+    y, tro, _ = run_wg_stack(x, p["w_qkvg"], p["w_o"], p["w_r"], wwg, w.H, "f32", attnres_block=0)
+    yref, tr = O.stack(x, p["w_qkvg"], p["w_o"], p["w_r"], w.H, attnres_block=0, keep_trace=True,
+                       w_wg=wwg)
+    for l in range(w.L):
+        assert_close(tro[l], tr["o"][l], "f32", f"o_{l + 1}")
+    assert_close(y - x, yref - x, "f32", "y - x")
+
+
+def test_stack_bf16_zero_write_gate_weights_double_eps():
+    # W_wg = 0: every gate is sigmoid(0) = 1/2, which only doubles eps. eps is
+    # set near the denominators phi(Q).z (about 300 keys x 20) so it matters.
+    x, wq, wo, wr, H = small_bf16_stack(8, N=300, seed=94)
+    zeros = [np.zeros((H, x.shape[-1]), np.float32) for _ in range(8)]
+    y_wg, _, _ = run_wg_stack(x, wq, wo, wr, zeros, H, "bf16", eps=3000.0)
+    y_2e, _, _ = run_stack(x, wq, wo, wr, H, "bf16", eps=6000.0)
+    y_1e, _, _ = run_stack(x, wq, wo, wr, H, "bf16", eps=3000.0)
+    assert rel_l2(y_wg - x, y_2e - x) < 2e-3
+    assert rel_l2(y_1e - x, y_2e - x) > 2e-2
 
 
 def test_stack_bf16_single_block_attnres_on_equals_off():

@@ -92,6 +92,8 @@ STACKS: Dict[str, StackWorkload] = {w.name: w for w in (HYBRID4_F32, STACK480P, 
 # tags of the per-tensor streams
 TAG_X, TAG_Q, TAG_K, TAG_V, TAG_G, TAG_WR = 0, 10, 11, 12, 13, 300
 TAG_WQKVG, TAG_WO = 100, 200
+TAG_WGATE = 14        # write-gate logits [B, N, H] of an isolated linear layer
+TAG_WWG = 400         # write-gate projection weights W_wg[l] [H, D] (tag 400 + l)
 
 
 # ---------------------------------------------------------------------------

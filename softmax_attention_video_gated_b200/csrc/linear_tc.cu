@@ -298,12 +298,30 @@ __global__ void __launch_bounds__(256) lin_reduce_bf16_kernel(const float* __res
   const int elems = HD * HD + HD;
   const float* p = partial + bh * n_chunks * elems;
   __nv_bfloat16* o = state_op + bh * STATE_ROWS * HD;
+  if (n_chunks <= 8) {
+    // all 4 x n_chunks loads issued before any add (latency, not bandwidth, bounds this)
+    float v[4][8];
 #pragma unroll
-  for (int r = 0; r < 4; ++r) {
-    const int k = ki * 32 + ty + 8 * r, n = ni * 32 + tx;
-    float acc = 0.f;
-    for (int c = 0; c < n_chunks; ++c) acc += p[static_cast<int64_t>(c) * elems + k * HD + n];
-    tile[ty + 8 * r][tx] = acc;
+    for (int r = 0; r < 4; ++r) {
+      const float* pp = p + (ki * 32 + ty + 8 * r) * HD + ni * 32 + tx;
+#pragma unroll
+      for (int c = 0; c < 8; ++c) v[r][c] = c < n_chunks ? pp[static_cast<int64_t>(c) * elems] : 0.f;
+    }
+#pragma unroll
+    for (int r = 0; r < 4; ++r) {
+      float acc = 0.f;
+#pragma unroll
+      for (int c = 0; c < 8; ++c) acc += v[r][c];
+      tile[ty + 8 * r][tx] = acc;
+    }
+  } else {
+#pragma unroll
+    for (int r = 0; r < 4; ++r) {
+      const int k = ki * 32 + ty + 8 * r, n = ni * 32 + tx;
+      float acc = 0.f;
+      for (int c = 0; c < n_chunks; ++c) acc += p[static_cast<int64_t>(c) * elems + k * HD + n];
+      tile[ty + 8 * r][tx] = acc;
+    }
   }
   __syncthreads();
 #pragma unroll

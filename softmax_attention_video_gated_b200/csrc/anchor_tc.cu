@@ -23,13 +23,20 @@
 // and the commit that reports S_{j+1} also covers P_j V_j, so a softmax warp
 // that sees S_{j+1} may rescale O.
 // Softmax per row: running max in the log2 domain, rescaled only when it grows
-// by more than 8 (p <= 2^8 otherwise, exact after the final 1/l); one FFMA per
-// element folds the scale. Exponentials run on the MUFU unit; kPolyEvery can
-// send every k-th one to the FMA pipe instead (Cody-Waite reduction and a
-// minimax cubic, see fit_exp2_poly.py). Measured on B200 at 720p: all-MUFU
-// 4.37 ms, one in four on the FMA pipe 4.77 ms, one in two 5.26 ms, and no
-// exponentials at all 4.26 ms -- this kernel is bound by its MMA pipeline
-// (3.54 ms with an empty softmax), not by the exponentials.
+// by more than 8 (p <= 2^8 otherwise, exact after the final 1/l); the max uses
+// three-input max, and the scale-and-shift and the row sum run on packed fp32
+// pairs (one f32x2 FFMA or FADD per two keys). Exponentials run on the MUFU
+// unit; kPolyEvery can send every k-th one to the FMA pipe instead (Cody-Waite
+// reduction and a minimax cubic, see fit_exp2_poly.py).
+// What bounds it (720p layer on B200, clock64 traces of one CTA): the softmax
+// warps wait for S about half of each 128-key step; the MMA thread issues
+// without pause, each 128x128x16 MMA taking ~88 cycles with both operands in
+// shared memory and ~59 with P in TMEM, and the tensor pipe drains while that
+// thread waits on barriers between MMA groups. Measured: 4.02 ms with packed
+// pairs, 4.35 ms without; sending one exponential pair in eight, four or three
+// to the FMA pipe: 4.10, 4.33, 4.52 ms; MMAs alone (no softmax dependency):
+// 3.10 ms. The wait for K_{j+1} sits after the first tile's P V issue so it
+// overlaps that MMA.
 #include <algorithm>
 #include <math.h>
 
@@ -246,9 +253,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         const bool more = j + 1 < nkv;
         const int kn = (j + 1) % K_STAGES;
         if (!mbar_wait(&tl->v_full[j % V_STAGES], (j / V_STAGES) & 1, abort_flag, status,
-                       WHERE_ANCHOR) ||
-            (more && !mbar_wait(&tl->k_full[kn], ((j + 1) / K_STAGES) & 1, abort_flag, status,
-                                WHERE_ANCHOR))) {
+                       WHERE_ANCHOR)) {
           ok = false;
           break;
         }
@@ -260,6 +265,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           tc_fence_after();
           issue_pv(t, j);
           if (t == ntiles - 1) umma_commit(&tl->v_empty[j % V_STAGES]);
+          // K_{j+1} is first needed here: this wait overlaps the P V just issued
+          if (t == 0 && more &&
+              !mbar_wait(&tl->k_full[kn], ((j + 1) / K_STAGES) & 1, abort_flag, status,
+                         WHERE_ANCHOR)) {
+            ok = false;
+            break;
+          }
           if (more) {
             issue_s(t, j + 1);
             if (t == ntiles - 1) umma_commit(&tl->k_empty[kn]);
@@ -305,13 +317,19 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           for (int i = 0; i < BKV; ++i)
             if (i >= valid) s[i] = -INFINITY;
         }
+        // row max: eight chains of three-input max over the 128 keys
         float mx8[8];
 #pragma unroll
-        for (int i = 0; i < 8; ++i) mx8[i] = s[i];
+        for (int k = 0; k < 8; ++k) mx8[k] = max3_f(s[k], s[k + 8], s[k + 16]);
 #pragma unroll
-        for (int i = 8; i < BKV; ++i) mx8[i & 7] = fmaxf(mx8[i & 7], s[i]);
-        const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
-                               fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7]))) *
+        for (int base = 24; base + 16 <= BKV - 8; base += 16)
+#pragma unroll
+          for (int k = 0; k < 8; ++k) mx8[k] = max3_f(mx8[k], s[base + k], s[base + 8 + k]);
+#pragma unroll
+        for (int k = 0; k < 8; ++k) mx8[k] = fmaxf(mx8[k], s[BKV - 8 + k]);
+        const float mx = fmaxf(max3_f(max3_f(mx8[0], mx8[1], mx8[2]),
+                                      max3_f(mx8[3], mx8[4], mx8[5]), mx8[6]),
+                               mx8[7]) *
                          scale_log2;
         const bool grow = mx > m + kRescaleThreshold;
         float factor = 1.f;
@@ -333,26 +351,32 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           }
         }
         l *= factor;
-        const float neg_m = -m;
-        float acc[8];
+        // x = s * scale - m and the row sum on packed pairs (f32x2)
+        const uint64_t scale2 = f2pack(scale_log2, scale_log2), negm2 = f2pack(-m, -m);
+        uint64_t acc2[4];
 #pragma unroll
-        for (int i = 0; i < 8; ++i) acc[i] = 0.f;
+        for (int i = 0; i < 4; ++i) acc2[i] = f2pack(0.f, 0.f);
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
           uint32_t pk[16];
 #pragma unroll
           for (int i = 0; i < 16; ++i) {
-            const float x0 = fmaf(s[32 * c + 2 * i], scale_log2, neg_m);
-            const float x1 = fmaf(s[32 * c + 2 * i + 1], scale_log2, neg_m);
+            float x0, x1;
+            f2unpack(fma_f2(f2pack(s[32 * c + 2 * i], s[32 * c + 2 * i + 1]), scale2, negm2), x0,
+                     x1);
             const float p0 = ex2_row<kPolyEvery>(x0, 2 * i);
             const float p1 = ex2_row<kPolyEvery>(x1, 2 * i + 1);
-            acc[i & 7] += p0 + p1;
+            acc2[i & 3] = add_f2(acc2[i & 3], f2pack(p0, p1));
             pk[i] = pack_bf16x2(p0, p1);
           }
           tmem_st16(s_col + 16 * c, pk);
         }
         tmem_wait_st();
-        l += ((acc[0] + acc[1]) + (acc[2] + acc[3])) + ((acc[4] + acc[5]) + (acc[6] + acc[7]));
+        {
+          float u0, u1;
+          f2unpack(add_f2(add_f2(acc2[0], acc2[1]), add_f2(acc2[2], acc2[3])), u0, u1);
+          l += u0 + u1;
+        }
         tc_fence_before();
         mbar_arrive(&tl->p_full[t]);
       }

@@ -18,11 +18,12 @@
 //  2. lin_reduce: sums the chunk partials in chunk order (deterministic) and
 //     writes the read-out operand [S^T | z_hi | z_lo | 0] as bf16 [144 x 128]
 //     (z split in two bf16 rows keeps it to ~16 bits).
-//  3. lin_readout_tc: one CTA per 128-token tile. TMA loads Q, G and the
-//     state operand; ReLU on Q in shared memory; one M=128, N=144, K=128 MMA
-//     gives the numerator (columns 0..127) and denominator (columns 128, 129)
-//     together; the epilogue divides, applies the sigmoid gate and residual,
-//     and writes Y through a TMA store.
+//  3. lin_readout_tc: persistent over the same chunks as the state pass. The
+//     state operand is loaded once; Q and G tiles stream through a 2-stage
+//     TMA ring; one M=128, N=144, K=128 MMA per tile gives the numerator
+//     (columns 0..127) and denominator (columns 128, 129) together into one of
+//     two TMEM accumulators; eight epilogue warps divide, apply the sigmoid
+//     gate and residual, and write Y through per-warp TMA stores.
 #include <algorithm>
 
 #include "common.cuh"
@@ -343,42 +344,69 @@ __global__ void __launch_bounds__(256) lin_reduce_bf16_kernel(const float* __res
 }
 
 // ------------------------------------------------------------------ read-out
+// Persistent over the state pass's chunks (one CTA per (token chunk, head,
+// batch), one wave). The head's read-out operand [S^T | z_hi | z_lo | 0] is
+// loaded once; 128-token tiles of Q and G stream through a 2-stage TMA ring.
+// One M=128, N=144, K=128 MMA per tile gives numerator (columns 0..127) and
+// denominator (128, 129) into one of two TMEM accumulators, so the MMA of the
+// next tile runs during this tile's epilogue. Eight epilogue warps: warp w
+// owns TMEM lane quadrant w % 4 (32 rows) and one 64-column half; each thread
+// applies ReLU to its half-row of Q when the producer has not, and finishes
+// its half-row of Y (divide, sigmoid(G), residual) into its warp's staging
+// slot, which the warp stores by TMA. No barrier spans more than one warp
+// inside the tile loop; a warp waits for its own previous store only before
+// it reuses its slot.
+constexpr int RO_STAGES = 2;
+constexpr int RO_STAGE_BYTES = 4 * BOX_BYTES;          // Q (2 boxes) + G (2 boxes)
+constexpr int RO_G = 2 * BOX_BYTES;                    // G's offset in a stage
+constexpr int RO_S_OFF = RO_STAGES * RO_STAGE_BYTES;   // the state operand: 2 x [64 x 144]
+constexpr int RO_Y_OFF = RO_S_OFF + 2 * STATE_BOX_BYTES;
+constexpr int RO_Y_SLOT = 32 * 128;                    // one warp's [64 x 32] bf16 slot
+constexpr int RO_TAIL_OFF = RO_Y_OFF + 8 * RO_Y_SLOT;
+constexpr int RO_THREADS = 320;                        // producer, MMA, 8 epilogue warps
 struct ReadoutTail {
-  uint64_t full_qs;
-  uint64_t full_g;
-  uint64_t relu_done;
-  uint64_t acc_full;
+  uint64_t full[RO_STAGES];
+  uint64_t relu_done[RO_STAGES];
+  uint64_t empty[RO_STAGES];
+  uint64_t acc_full[2];
+  uint64_t acc_empty[2];
+  uint64_t s_full;
   uint64_t drain;
   uint32_t tmem_base;
   int abort_flag;
 };
-constexpr int RO_Q_OFF = 0;                                   // 32 KB, reused for Y
-constexpr int RO_G_OFF = 2 * BOX_BYTES;                       // 32 KB
-constexpr int RO_S_OFF = 4 * BOX_BYTES;                       // 36 KB
-constexpr int RO_TAIL_OFF = RO_S_OFF + 2 * STATE_BOX_BYTES;
 constexpr size_t kReadoutSmem = 1024 + RO_TAIL_OFF + sizeof(ReadoutTail);
-constexpr int RO_TMEM_COLS = 256;
+constexpr int RO_TMEM_COLS = 512;                      // two 256-column accumulators
 
-__global__ void __launch_bounds__(192)
+__global__ void __launch_bounds__(RO_THREADS, 1)
     lin_readout_tc_kernel(const __grid_constant__ CUtensorMap map_q,
                           const __grid_constant__ CUtensorMap map_g,
                           const __grid_constant__ CUtensorMap map_s,
-                          const __grid_constant__ CUtensorMap map_o, int N, int H, float eps,
-                          unsigned flags, const __nv_bfloat16* residual, int64_t ldr,
-                          int* status) {
+                          const __grid_constant__ CUtensorMap map_o, int N, int H,
+                          int tiles_per_chunk, float eps, unsigned flags,
+                          const __nv_bfloat16* residual, int64_t ldr, int* status) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
   ReadoutTail* tl = reinterpret_cast<ReadoutTail*>(smem + RO_TAIL_OFF);
-  const int tile = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
-  const int t0 = tile * TT;
+  const int c = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
   const int warp = warp_id(), lane = lane_id();
+  const int tiles_total = (N + TT - 1) / TT;
+  const int tile0 = c * tiles_per_chunk;
+  const int ntiles = max(0, min(tiles_per_chunk, tiles_total - tile0));
+  const bool features = (flags & SVA_FLAG_QK_FEATURES) != 0;
 
   if (threadIdx.x == 0) {
-    mbar_init(&tl->full_qs, 1);
-    mbar_init(&tl->full_g, 1);
-    mbar_init(&tl->relu_done, 128);
-    mbar_init(&tl->acc_full, 1);
+    for (int st = 0; st < RO_STAGES; ++st) {
+      mbar_init(&tl->full[st], 1);
+      mbar_init(&tl->relu_done[st], 256);
+      mbar_init(&tl->empty[st], 8);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&tl->acc_full[a], 1);
+      mbar_init(&tl->acc_empty[a], 8);
+    }
+    mbar_init(&tl->s_full, 1);
     mbar_init(&tl->drain, 1);
     tl->abort_flag = 0;
     fence_mbar_init();
@@ -394,129 +422,182 @@ __global__ void __launch_bounds__(192)
   volatile int* abort_flag = &tl->abort_flag;
 
   if (warp == 0) {
-    if (lane == 0) {
+    if (lane == 0 && ntiles > 0) {
+      // ------------------------------------------------ TMA producer
       const int srow = (b * H + h) * STATE_ROWS;
-      mbar_arrive_expect_tx(&tl->full_qs, 2 * BOX_BYTES + 2 * STATE_BOX_BYTES);
-      tma_load_3d(&map_q, &tl->full_qs, smem + RO_Q_OFF, h * HD, t0, b);
-      tma_load_3d(&map_q, &tl->full_qs, smem + RO_Q_OFF + BOX_BYTES, h * HD + 64, t0, b);
-      tma_load_2d(&map_s, &tl->full_qs, smem + RO_S_OFF, 0, srow);
-      tma_load_2d(&map_s, &tl->full_qs, smem + RO_S_OFF + STATE_BOX_BYTES, 64, srow);
-      mbar_arrive_expect_tx(&tl->full_g, 2 * BOX_BYTES);
-      tma_load_3d(&map_g, &tl->full_g, smem + RO_G_OFF, h * HD, t0, b);
-      tma_load_3d(&map_g, &tl->full_g, smem + RO_G_OFF + BOX_BYTES, h * HD + 64, t0, b);
-      // both barriers are waited on below by the epilogue threads before exit,
-      // (bounded), so no load is left in flight when the CTA finishes
+      mbar_arrive_expect_tx(&tl->s_full, 2 * STATE_BOX_BYTES);
+      tma_load_2d(&map_s, &tl->s_full, smem + RO_S_OFF, 0, srow);
+      tma_load_2d(&map_s, &tl->s_full, smem + RO_S_OFF + STATE_BOX_BYTES, 64, srow);
+      int stage = 0;
+      uint32_t phase = 0;
+      int issued = 0;
+      bool ok = true;
+      for (int i = 0; i < ntiles; ++i) {
+        if (!mbar_wait(&tl->empty[stage], phase ^ 1, abort_flag, status, WHERE_LIN_READOUT)) {
+          ok = false;
+          break;
+        }
+        uint8_t* sb = smem + stage * RO_STAGE_BYTES;
+        const int t0 = (tile0 + i) * TT;
+        mbar_arrive_expect_tx(&tl->full[stage], RO_STAGE_BYTES);
+        tma_load_3d(&map_q, &tl->full[stage], sb, h * HD, t0, b);
+        tma_load_3d(&map_q, &tl->full[stage], sb + BOX_BYTES, h * HD + 64, t0, b);
+        tma_load_3d(&map_g, &tl->full[stage], sb + RO_G, h * HD, t0, b);
+        tma_load_3d(&map_g, &tl->full[stage], sb + RO_G + BOX_BYTES, h * HD + 64, t0, b);
+        ++issued;
+        if (++stage == RO_STAGES) {
+          stage = 0;
+          phase ^= 1;
+        }
+      }
+      (void)drain_wait(&tl->s_full, 0);
+      if (!ok)
+        for (int i = max(0, issued - RO_STAGES); i < issued; ++i)
+          (void)drain_wait(&tl->full[i % RO_STAGES], (i / RO_STAGES) & 1);
     }
   } else if (warp == 1) {
-    if (lane == 0) {
+    if (lane == 0 && ntiles > 0) {
+      // ------------------------------------------------ MMA issuer
       constexpr uint32_t idesc = idesc_bf16_f32(128, STATE_ROWS, false, false);
-      if (mbar_wait(&tl->relu_done, 0, abort_flag, status, WHERE_LIN_READOUT)) {
+      bool ok = mbar_wait(&tl->s_full, 0, abort_flag, status, WHERE_LIN_READOUT);
+      const uint32_t saddr = smem_u32(smem + RO_S_OFF);
+      int stage = 0;
+      uint32_t phase = 0;
+      for (int i = 0; i < ntiles && ok; ++i) {
+        const int acc = i & 1;
+        const uint32_t acc_phase = (i >> 1) & 1;
+        // Q is ready once loaded (features) or once the epilogue applied ReLU
+        uint64_t* ready = features ? &tl->full[stage] : &tl->relu_done[stage];
+        if (!mbar_wait(ready, phase, abort_flag, status, WHERE_LIN_READOUT) ||
+            !mbar_wait(&tl->acc_empty[acc], acc_phase ^ 1, abort_flag, status,
+                       WHERE_LIN_READOUT)) {
+          ok = false;
+          break;
+        }
         tc_fence_after();
-        const uint32_t qaddr = smem_u32(smem + RO_Q_OFF);
-        const uint32_t saddr = smem_u32(smem + RO_S_OFF);
+        const uint32_t qaddr = smem_u32(smem + stage * RO_STAGE_BYTES);
 #pragma unroll
         for (int kk = 0; kk < HD / 16; ++kk) {
           const int bx = kk >> 2, w = kk & 3;
           const uint64_t ad = smem_desc(qaddr + bx * BOX_BYTES + w * 32, 16, 1024);
           const uint64_t bd = smem_desc(saddr + bx * STATE_BOX_BYTES + w * 32, 16, 1024);
-          umma_ss(tmem, ad, bd, idesc, kk != 0 ? 1u : 0u);
+          umma_ss(tmem + acc * 256, ad, bd, idesc, kk != 0 ? 1u : 0u);
         }
-        umma_commit(&tl->acc_full);
+        umma_commit(&tl->acc_full[acc]);
+        if (++stage == RO_STAGES) {
+          stage = 0;
+          phase ^= 1;
+        }
       }
       umma_commit(&tl->drain);
       (void)drain_wait(&tl->drain, 0);
     }
-  } else {
-    const int wt = threadIdx.x - 64;
-    const int q = warp & 3;
-    bool ok;
-    {
-      // ReLU on the Q tile, in place
-      bool w = mbar_wait(&tl->full_qs, 0, abort_flag, status, WHERE_LIN_READOUT);
-      ok = __all_sync(0xffffffffu, w);
-      if (ok && (flags & SVA_FLAG_QK_FEATURES) == 0) {
-        const int ch = wt & 15, rc = wt >> 4;
-        const int box = ch >> 3, cl = ch & 7;
-        uint8_t* qt = smem + RO_Q_OFF + box * BOX_BYTES + ((cl ^ rc) << 4);
-#pragma unroll 4
-        for (int j = 0; j < TT / 8; ++j) {
-          uint4* p = reinterpret_cast<uint4*>(qt + (rc + 8 * j) * 128);
-          uint4 v = *p;
-          v.x = relu_bf16x2(v.x);
-          v.y = relu_bf16x2(v.y);
-          v.z = relu_bf16x2(v.z);
-          v.w = relu_bf16x2(v.w);
-          *p = v;
-        }
-        fence_proxy_async_smem();
-      }
-      if (ok) mbar_arrive(&tl->relu_done);
-    }
-    if (ok) {
-      bool w = mbar_wait(&tl->acc_full, 0, abort_flag, status, WHERE_LIN_READOUT);
-      w = w && mbar_wait(&tl->full_g, 0, abort_flag, status, WHERE_LIN_READOUT);
-      ok = __all_sync(0xffffffffu, w);
-    }
-    if (ok) {
-      tc_fence_after();
-      const int r = q * 32 + lane;                 // row of the tile = TMEM lane
-      const uint32_t trow = tmem + (static_cast<uint32_t>(q * 32) << 16);
-      uint32_t dd[16];
-      tmem_ld16(trow + HD, dd);
-      tmem_wait_ld();
-      const float inv = 1.0f / (__uint_as_float(dd[0]) + __uint_as_float(dd[1]) + eps);
-      const int t = t0 + r;
-      const bool row_ok = t < N;
-      const __nv_bfloat16* res =
-          (residual != nullptr && row_ok)
-              ? residual + (static_cast<int64_t>(b) * N + t) * ldr + h * HD
-              : nullptr;
-#pragma unroll 1
-      for (int cc = 0; cc < HD; cc += 32) {
-        uint32_t num[32];
-        tmem_ld32(trow + cc, num);
-        tmem_wait_ld();
-        const int box = cc >> 6;
+  } else if (ntiles > 0) {
+    // ------------------------------------------------ epilogue: half a row per thread
+    const int ew = warp - 2;                 // epilogue warp 0..7
+    const int wq = warp & 3;                 // TMEM lane quadrant of this warp
+    const int half = ew >> 2;                // 64-column half of the tile
+    const int r = wq * 32 + lane;            // row of the tile
+    const uint32_t lane_base = static_cast<uint32_t>(wq * 32) << 16;
+    uint8_t* yslot = smem + RO_Y_OFF + ew * RO_Y_SLOT;
+    // ReLU on this thread's half-row of Q in tile k (its stage), then report it
+    auto relu_tile = [&](int k) -> bool {
+      const int st = k % RO_STAGES;
+      const bool w = mbar_wait(&tl->full[st], (k / RO_STAGES) & 1, abort_flag, status,
+                               WHERE_LIN_READOUT);
+      if (!__all_sync(0xffffffffu, w)) return false;
+      uint8_t* qrow = smem + st * RO_STAGE_BYTES + half * BOX_BYTES + r * 128;
 #pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          const int cl = ((cc & 63) >> 3) + k;
-          const uint32_t off = box * BOX_BYTES + r * 128 + ((cl ^ (r & 7)) << 4);
-          const uint4 gv = *reinterpret_cast<const uint4*>(smem + RO_G_OFF + off);
-          float gg[8] = {bf16lo_to_f32(gv.x), bf16hi_to_f32(gv.x), bf16lo_to_f32(gv.y),
-                         bf16hi_to_f32(gv.y), bf16lo_to_f32(gv.z), bf16hi_to_f32(gv.z),
-                         bf16lo_to_f32(gv.w), bf16hi_to_f32(gv.w)};
-          float y[8];
-#pragma unroll
-          for (int e = 0; e < 8; ++e)
-            y[e] = __uint_as_float(num[8 * k + e]) * inv * fast_sigmoid(gg[e]);
-          if (res != nullptr) {
-            const uint4 rv = *reinterpret_cast<const uint4*>(res + cc + 8 * k);
-            y[0] += bf16lo_to_f32(rv.x); y[1] += bf16hi_to_f32(rv.x);
-            y[2] += bf16lo_to_f32(rv.y); y[3] += bf16hi_to_f32(rv.y);
-            y[4] += bf16lo_to_f32(rv.z); y[5] += bf16hi_to_f32(rv.z);
-            y[6] += bf16lo_to_f32(rv.w); y[7] += bf16hi_to_f32(rv.w);
-          }
-          uint4 o;
-          o.x = pack_bf16x2(y[0], y[1]);
-          o.y = pack_bf16x2(y[2], y[3]);
-          o.z = pack_bf16x2(y[4], y[5]);
-          o.w = pack_bf16x2(y[6], y[7]);
-          *reinterpret_cast<uint4*>(smem + RO_Q_OFF + off) = o;
-        }
+      for (int cl = 0; cl < 8; ++cl) {
+        uint4* p = reinterpret_cast<uint4*>(qrow + ((cl ^ (r & 7)) << 4));
+        uint4 v = *p;
+        v.x = relu_bf16x2(v.x);
+        v.y = relu_bf16x2(v.y);
+        v.z = relu_bf16x2(v.z);
+        v.w = relu_bf16x2(v.w);
+        *p = v;
       }
       fence_proxy_async_smem();
-    } else {
-      // make sure no TMA load is still writing shared memory before exit
-      (void)drain_wait(&tl->full_qs, 0);
-      (void)drain_wait(&tl->full_g, 0);
+      mbar_arrive(&tl->relu_done[st]);
+      return true;
+    };
+    bool ok = features || relu_tile(0);
+    for (int i = 0; i < ntiles && ok; ++i) {
+      const int st = i % RO_STAGES, acc = i & 1;
+      const uint32_t phase = (i / RO_STAGES) & 1, acc_phase = (i >> 1) & 1;
+      const int t0 = (tile0 + i) * TT;
+      {
+        bool w = mbar_wait(&tl->full[st], phase, abort_flag, status, WHERE_LIN_READOUT);
+        w = w && mbar_wait(&tl->acc_full[acc], acc_phase, abort_flag, status, WHERE_LIN_READOUT);
+        if (!__all_sync(0xffffffffu, w)) {
+          ok = false;
+          break;
+        }
+      }
+      tc_fence_after();
+      const uint32_t trow = tmem + lane_base + acc * 256;
+      uint32_t dd[16], num0[32], num1[32];
+      tmem_ld16(trow + HD, dd);
+      tmem_ld32(trow + half * 64, num0);
+      tmem_ld32(trow + half * 64 + 32, num1);
+      tmem_wait_ld();
+      // the accumulator is read: hand it back to the MMA
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&tl->acc_empty[acc]);
+      const float inv = 1.0f / (__uint_as_float(dd[0]) + __uint_as_float(dd[1]) + eps);
+      // this warp's previous store has read its slot before the slot is rewritten
+      if (lane == 0) tma_store_wait_read0();
+      __syncwarp();
+      const int t = t0 + r;
+      const __nv_bfloat16* res =
+          (residual != nullptr && t < N)
+              ? residual + (static_cast<int64_t>(b) * N + t) * ldr + h * HD + half * 64
+              : nullptr;
+      const uint8_t* grow = smem + st * RO_STAGE_BYTES + RO_G + half * BOX_BYTES + r * 128;
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        const uint4 gv = *reinterpret_cast<const uint4*>(grow + ((k ^ (r & 7)) << 4));
+        const float gg[8] = {bf16lo_to_f32(gv.x), bf16hi_to_f32(gv.x), bf16lo_to_f32(gv.y),
+                             bf16hi_to_f32(gv.y), bf16lo_to_f32(gv.z), bf16hi_to_f32(gv.z),
+                             bf16lo_to_f32(gv.w), bf16hi_to_f32(gv.w)};
+        float y[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e)
+          y[e] = __uint_as_float(k < 4 ? num0[8 * k + e] : num1[8 * (k - 4) + e]) * inv *
+                 fast_sigmoid(gg[e]);
+        if (res != nullptr) {
+          const uint4 rv = *reinterpret_cast<const uint4*>(res + 8 * k);
+          y[0] += bf16lo_to_f32(rv.x); y[1] += bf16hi_to_f32(rv.x);
+          y[2] += bf16lo_to_f32(rv.y); y[3] += bf16hi_to_f32(rv.y);
+          y[4] += bf16lo_to_f32(rv.z); y[5] += bf16hi_to_f32(rv.z);
+          y[6] += bf16lo_to_f32(rv.w); y[7] += bf16hi_to_f32(rv.w);
+        }
+        uint4 o;
+        o.x = pack_bf16x2(y[0], y[1]);
+        o.y = pack_bf16x2(y[2], y[3]);
+        o.z = pack_bf16x2(y[4], y[5]);
+        o.w = pack_bf16x2(y[6], y[7]);
+        *reinterpret_cast<uint4*>(yslot + lane * 128 + ((k ^ (lane & 7)) << 4)) = o;
+      }
+      // G of this stage is read: release it (the MMA finished with Q at acc_full)
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&tl->empty[st]);
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0 && t0 + wq * 32 < N) {
+        tma_store_3d(&map_o, yslot, h * HD + half * 64, t0 + wq * 32, b);
+        tma_store_commit();
+      }
+      // the next tile's ReLU after this epilogue: its load was issued when the
+      // previous epilogue released the stage, so it has had this epilogue to land
+      if (!features && i + 1 < ntiles && !relu_tile(i + 1)) {
+        ok = false;
+        break;
+      }
     }
-    named_barrier_sync(1, 128);
-    if (ok && wt == 0) {
-      tma_store_3d(&map_o, smem + RO_Q_OFF, h * HD, t0, b);
-      tma_store_3d(&map_o, smem + RO_Q_OFF + BOX_BYTES, h * HD + 64, t0, b);
-      tma_store_commit();
-      tma_store_wait_read0();
-    }
+    // the slot stays valid until this warp's last store has read it
+    if (lane == 0) tma_store_wait_read0();
   }
 
   tc_fence_before();
@@ -573,9 +654,19 @@ cudaError_t linear_bf16(const sva_attn_args& a, int* status, void* scratch, cuda
   const int D = a.H * a.d;
   CUtensorMap mk, mv, mq, mg, mo, ms;
   if (!act_map(&mk, a.k, a.ldk, a.B, a.N, D) || !act_map(&mv, a.v, a.ldv, a.B, a.N, D) ||
-      !act_map(&mq, a.q, a.ldq, a.B, a.N, D) || !act_map(&mg, a.gate, a.ldg, a.B, a.N, D) ||
-      !act_map(&mo, a.out, a.ldo, a.B, a.N, D))
+      !act_map(&mq, a.q, a.ldq, a.B, a.N, D) || !act_map(&mg, a.gate, a.ldg, a.B, a.N, D))
     return cudaErrorInvalidValue;
+  {
+    // Y: one [64 x 32] box per epilogue warp
+    const uint64_t dims[3] = {static_cast<uint64_t>(D), static_cast<uint64_t>(a.N),
+                              static_cast<uint64_t>(a.B)};
+    const uint64_t strides[2] = {static_cast<uint64_t>(a.ldo) * 2,
+                                 static_cast<uint64_t>(a.ldo) * 2 * static_cast<uint64_t>(a.N)};
+    const uint32_t box[3] = {64, 32, 1};
+    if (!encode_tmap(&mo, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, a.out, dims, strides, box,
+                     CU_TENSOR_MAP_SWIZZLE_128B))
+      return cudaErrorInvalidValue;
+  }
   {
     const uint64_t dims[2] = {HD, static_cast<uint64_t>(a.B) * a.H * STATE_ROWS};
     const uint64_t strides[1] = {HD * 2};
@@ -607,10 +698,9 @@ cudaError_t linear_bf16(const sva_attn_args& a, int* status, void* scratch, cuda
   e = cudaFuncSetAttribute(lin_readout_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            static_cast<int>(kReadoutSmem));
   if (e != cudaSuccess) return e;
-  dim3 grid((a.N + TT - 1) / TT, a.H, a.B);
-  lin_readout_tc_kernel<<<grid, 192, kReadoutSmem, s>>>(
-      mq, mg, ms, mo, a.N, a.H, a.eps, a.flags, static_cast<const __nv_bfloat16*>(a.residual),
-      a.ldr, status);
+  lin_readout_tc_kernel<<<dim3(p.n_chunks, a.H, a.B), RO_THREADS, kReadoutSmem, s>>>(
+      mq, mg, ms, mo, a.N, a.H, p.tiles_per_chunk, a.eps, a.flags,
+      static_cast<const __nv_bfloat16*>(a.residual), a.ldr, status);
   return cudaGetLastError();
 }
 

@@ -431,6 +431,16 @@ def run_case(args):
         ws = sva.workspace(256)
         fn = lambda: sva.sva_projection_fwd(x, w, y, ws=ws)  # noqa: E731
         work, unit = 2.0 * M * K * Nout, "TFLOP/s"
+    elif args.case == "route":
+        # AttnRes router of a linear layer in block nb + 1: u = h + sum_b alpha_b s_b
+        M, nb = B * N, args.nb
+        hs = W.normal_torch((M, D), 1.0, seed, W.TAG_X, "f32")
+        ks = [W.normal_torch((M, D), 1.0, seed, 901 + i, "bf16") for i in range(nb)]
+        ss = [W.normal_torch((M, D), 1.0, seed, 911 + i, "bf16") for i in range(nb)]
+        u = torch.empty(M, D, device="cuda", dtype=torch.bfloat16)
+        ws = sva.workspace(256)
+        fn = lambda: sva.sva_attnres_route(hs, ks, ss, u)  # noqa: E731
+        work, unit = (4.0 + 4.0 * nb + 2.0) * M * D, "GB/s"
     else:  # proj_out: h += x W_o^T with the bf16 copy of h, as in the stack
         M, K, Nout = B * N, D, D
         x = W.normal_torch((M, K), 1.0, seed, W.TAG_X, "bf16")
@@ -517,7 +527,7 @@ def main():
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-all-softmax", action="store_true")
-    ap.add_argument("--case", choices=("anchor", "linear", "linear_wg", "gemm", "proj_out"),
+    ap.add_argument("--case", choices=("anchor", "linear", "linear_wg", "gemm", "proj_out", "route"),
                     help="time one kernel class alone instead of the stack")
     ap.add_argument("--sweep", action="store_true",
                     help="hybrid vs all-softmax 4-layer groups at 5 s .. 60 s of 720p video")
@@ -526,6 +536,7 @@ def main():
     ap.add_argument("--B", type=int, default=1)
     ap.add_argument("--N", type=int, default=19320)
     ap.add_argument("--H", type=int, default=24)
+    ap.add_argument("--nb", type=int, default=2, help="completed blocks the router mixes (--case route)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")

@@ -86,8 +86,8 @@ def algorithmic_work(kind: str, wl: dict, n_blocks_routed: int = 1):
 
     GEMMs: 2*M*K*N flops. Linear state pass: K and V read once (2*B*N*D*2 B).
     Linear read-out: Q and G read, Y written (3*B*N*D*2 B). Anchor: 4*B*N^2*D
-    flops (S = Q K^T and O = P V). Router: h (fp32) read, n_b keys and n_b
-    summaries read, u written."""
+    flops (S = Q K^T and O = P V). Router: h (fp32) read once, n_b keys and n_b
+    summaries read, u written: (4 + 4*n_b + 2)*B*N*D bytes."""
     B, N, D = wl["B"], wl["N"], wl["H"] * wl["d"]
     M = B * N
     if kind == "proj_qkvg":
@@ -389,11 +389,26 @@ def summarize(recs, steps, wl, peaks):
             e["achieved"] = work / (avg * 1e-3) / 1e12
             e["unit"] = "TFLOP/s"
             e["frac"] = e["achieved"] / peaks["bf16_tflops_sustained"]
-        elif bound == "hbm" and kind != "route":
+        elif bound == "hbm":
+            if kind == "route":
+                # routed layers mix 1, 2, ... completed blocks: total bytes over total time
+                work = sum(algorithmic_work("route", wl, nb)[1] for nb in routed_blocks(wl))
+                work /= max(1, len(routed_blocks(wl)))
             e["achieved"] = work / (avg * 1e-3) / 1e9
             e["unit"] = "GB/s"
             e["frac"] = e["achieved"] / peaks["hbm_gbs"]
         out[kind] = e
+    return out
+
+
+def routed_blocks(wl):
+    """Completed blocks each routed linear layer mixes, in layer order."""
+    out = []
+    blk, per = wl["attnres_block"], wl["softmax_period"]
+    for l in range(1, wl["L"] + 1):
+        c = (l + blk - 1) // blk if blk > 0 else 1
+        if blk > 0 and c >= 2 and not (per > 0 and l % per == 0):
+            out.append(c - 1)
     return out
 
 

@@ -131,6 +131,100 @@ __global__ void __launch_bounds__(256) route_kernel(const float* __restrict__ h,
   }
 }
 
+// bf16 router with one group of D / 8 threads per row (D a multiple of 256):
+// each thread keeps its 8 values of h in registers between the two steps, so h
+// is read from HBM once, and every load of a step is issued before any is
+// used (kept packed until then). The NB dot products are summed over the
+// group's warps through shared memory; several groups may share a CTA.
+template <int NB>
+__global__ void __launch_bounds__(512) route_rows_kernel(const float* __restrict__ h, RoutePtrs p,
+                                                         __nv_bfloat16* __restrict__ u,
+                                                         float* __restrict__ alpha, int64_t rows,
+                                                         int D, float inv_sqrt_d) {
+  __shared__ float part[16][NB];  // per-warp partial dots (at most 16 warps)
+  const int G = D >> 3;           // threads per row
+  const int g = threadIdx.x / G, tg = threadIdx.x - g * G;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t row = static_cast<int64_t>(blockIdx.x) * (blockDim.x / G) + g;
+  const bool valid = row < rows;
+  const int64_t off = (valid ? row : 0) * D + tg * 8;
+  float4 ha = make_float4(0.f, 0.f, 0.f, 0.f), hb = ha;
+  uint4 kq[NB];
+  if (valid) {
+    ha = *reinterpret_cast<const float4*>(h + off);
+    hb = *reinterpret_cast<const float4*>(h + off + 4);
+#pragma unroll
+    for (int b = 0; b < NB; ++b)
+      kq[b] = *reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(p.keys[b]) + off);
+  } else {
+#pragma unroll
+    for (int b = 0; b < NB; ++b) kq[b] = make_uint4(0u, 0u, 0u, 0u);
+  }
+  const float hv[8] = {ha.x, ha.y, ha.z, ha.w, hb.x, hb.y, hb.z, hb.w};
+#pragma unroll
+  for (int b = 0; b < NB; ++b) {
+    const uint32_t kw[4] = {kq[b].x, kq[b].y, kq[b].z, kq[b].w};
+    float d = 0.f;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      d = fmaf(hv[2 * i], bf16lo_to_f32(kw[i]), d);
+      d = fmaf(hv[2 * i + 1], bf16hi_to_f32(kw[i]), d);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) d += __shfl_xor_sync(0xffffffffu, d, o);
+    if (lane == 0) part[warp][b] = d;
+  }
+  __syncthreads();
+  // the group's warps are [g * G / 32, (g + 1) * G / 32); every thread sums them
+  const int w0 = (g * G) >> 5, nw = G >> 5;
+  float wts[NB];
+  float mx = -INFINITY;
+#pragma unroll
+  for (int b = 0; b < NB; ++b) {
+    float d = 0.f;
+    for (int w = 0; w < nw; ++w) d += part[w0 + w][b];
+    wts[b] = d * inv_sqrt_d;
+    mx = fmaxf(mx, wts[b]);
+  }
+  float sum = 0.f;
+#pragma unroll
+  for (int b = 0; b < NB; ++b) {
+    wts[b] = expf(wts[b] - mx);
+    sum += wts[b];
+  }
+  const float inv = 1.0f / sum;
+  if (!valid) return;
+  uint4 sq[NB];
+#pragma unroll
+  for (int b = 0; b < NB; ++b)
+    sq[b] = *reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(p.summaries[b]) + off);
+  float acc[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) acc[i] = hv[i];
+#pragma unroll
+  for (int b = 0; b < NB; ++b) {
+    const float wb = wts[b] * inv;
+    if (alpha != nullptr && tg == 0) alpha[row * NB + b] = wb;
+    const uint32_t sw[4] = {sq[b].x, sq[b].y, sq[b].z, sq[b].w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      acc[2 * i] = fmaf(wb, bf16lo_to_f32(sw[i]), acc[2 * i]);
+      acc[2 * i + 1] = fmaf(wb, bf16hi_to_f32(sw[i]), acc[2 * i + 1]);
+    }
+  }
+  Vec<__nv_bfloat16>::store(u + off, acc);
+}
+
+template <int NB>
+cudaError_t launch_route_rows(const float* h, const RoutePtrs& p, void* u, float* alpha,
+                              int64_t rows, int D, float inv_sqrt_d, cudaStream_t s) {
+  const int G = D / 8, per_cta = 512 / G;
+  const unsigned grid = static_cast<unsigned>((rows + per_cta - 1) / per_cta);
+  route_rows_kernel<NB><<<grid, G * per_cta, 0, s>>>(h, p, static_cast<__nv_bfloat16*>(u), alpha,
+                                                     rows, D, inv_sqrt_d);
+  return cudaGetLastError();
+}
+
 // ---------------------------------------------------------------------------
 // transpose (32 x 32 tiles through shared memory) and casts
 // ---------------------------------------------------------------------------
@@ -201,9 +295,18 @@ cudaError_t route(const float* h, const void* const* keys, const void* const* su
     p.keys[b] = keys[b];
     p.summaries[b] = summaries[b];
   }
+  const float inv_sqrt_d = 1.0f / sqrtf(static_cast<float>(D));
+  if (dt == SVA_BF16 && D % 256 == 0 && D / 8 <= 512) {
+    switch (n_blocks) {
+      case 1: return launch_route_rows<1>(h, p, u, alpha, rows, D, inv_sqrt_d, s);
+      case 2: return launch_route_rows<2>(h, p, u, alpha, rows, D, inv_sqrt_d, s);
+      case 3: return launch_route_rows<3>(h, p, u, alpha, rows, D, inv_sqrt_d, s);
+      case 4: return launch_route_rows<4>(h, p, u, alpha, rows, D, inv_sqrt_d, s);
+      default: break;  // more blocks: the warp-per-row kernel below
+    }
+  }
   const int warps = 8;
   const unsigned grid = static_cast<unsigned>((rows + warps - 1) / warps);
-  const float inv_sqrt_d = 1.0f / sqrtf(static_cast<float>(D));
   if (dt == SVA_BF16)
     route_kernel<__nv_bfloat16><<<grid, 32 * warps, 0, s>>>(
         h, p, n_blocks, static_cast<__nv_bfloat16*>(u), alpha, rows, D, inv_sqrt_d);

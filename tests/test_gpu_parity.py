@@ -246,10 +246,14 @@ def test_softmax_anchor_residual_in_place(dtype):
 # ------------------------------------------------------------------ AttnRes
 
 @pytest.mark.parametrize("dtype", ["bf16", "f32"])
-@pytest.mark.parametrize("nb", [1, 2, 3])
-def test_attnres_route(dtype, nb):
-    rng = np.random.default_rng(70 + nb)
-    rows, D = 1234, 384
+@pytest.mark.parametrize("nb", [1, 2, 3, 5])
+@pytest.mark.parametrize("D", [384, 512, 3072])
+def test_attnres_route(dtype, nb, D):
+    # D = 512 and 3072 take the bf16 row-group kernel (up to 4 blocks; 8 and 1
+    # rows per CTA, 1234 rows leaves a ragged last CTA); D = 384, 5 blocks and
+    # fp32 take the warp-per-row kernel
+    rng = np.random.default_rng(70 + nb + D)
+    rows = 1234
     h = rng.standard_normal((rows, D)).astype(np.float32)
     s = [W.round_to(rng.standard_normal((rows, D)).astype(np.float32), dtype) for _ in range(nb)]
     wr = W.round_to((rng.standard_normal((D, D)) / math.sqrt(D)).astype(np.float32), dtype)

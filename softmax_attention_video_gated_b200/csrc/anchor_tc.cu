@@ -35,8 +35,9 @@
 // thread waits on barriers between MMA groups. Measured: 4.02 ms with packed
 // pairs, 4.35 ms without; sending one exponential pair in eight, four or three
 // to the FMA pipe: 4.10, 4.33, 4.52 ms; MMAs alone (no softmax dependency):
-// 3.10 ms. The wait for K_{j+1} sits after the first tile's P V issue so it
-// overlaps that MMA.
+// 3.10 ms. The wait for K_{j+1} sat after the first tile's P V issue so it
+// overlaps that MMA; then 3.94 ms once the waits for V_j and K_{j+1} moved
+// from the MMA thread to a softmax warp of each tile.
 #include <algorithm>
 #include <math.h>
 
@@ -252,11 +253,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       for (int j = 0; j < nkv && ok; ++j) {
         const bool more = j + 1 < nkv;
         const int kn = (j + 1) % K_STAGES;
-        if (!mbar_wait(&tl->v_full[j % V_STAGES], (j / V_STAGES) & 1, abort_flag, status,
-                       WHERE_ANCHOR)) {
-          ok = false;
-          break;
-        }
+        // V_j and K_{j+1} need no wait here: a softmax warp of each tile saw
+        // them land before it reported P_j (its p_full arrival orders them)
         for (int t = 0; t < ntiles; ++t) {
           if (!mbar_wait(&tl->p_full[t], j & 1, abort_flag, status, WHERE_ANCHOR)) {
             ok = false;
@@ -265,13 +263,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           tc_fence_after();
           issue_pv(t, j);
           if (t == ntiles - 1) umma_commit(&tl->v_empty[j % V_STAGES]);
-          // K_{j+1} is first needed here: this wait overlaps the P V just issued
-          if (t == 0 && more &&
-              !mbar_wait(&tl->k_full[kn], ((j + 1) / K_STAGES) & 1, abort_flag, status,
-                         WHERE_ANCHOR)) {
-            ok = false;
-            break;
-          }
           if (more) {
             issue_s(t, j + 1);
             if (t == ntiles - 1) umma_commit(&tl->k_empty[kn]);
@@ -378,6 +369,20 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           l += u0 + u1;
         }
         tc_fence_before();
+        if (q == 0) {
+          // the MMA thread waits only for P: this warp checks that V_j and
+          // K_{j+1} are resident before P_j is reported (it has slack; the MMA
+          // thread's waits are on the critical path)
+          bool w = mbar_wait(&tl->v_full[j % V_STAGES], (j / V_STAGES) & 1, abort_flag, status,
+                             WHERE_ANCHOR);
+          if (j + 1 < nkv)
+            w = w && mbar_wait(&tl->k_full[(j + 1) % K_STAGES], ((j + 1) / K_STAGES) & 1,
+                               abort_flag, status, WHERE_ANCHOR);
+          if (!__all_sync(0xffffffffu, w)) {
+            ok = false;
+            break;
+          }
+        }
         mbar_arrive(&tl->p_full[t]);
       }
       if (ok && nkv > 0) {

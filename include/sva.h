@@ -240,6 +240,24 @@ size_t sva_hybrid_stack_workspace_bytes(const sva_stack_desc* desc);
 sva_status_t sva_hybrid_stack_fwd(const sva_stack_desc* desc, const void* x, void* y, void* ws,
                                   size_t ws_bytes, sva_stream_t stream);
 
+/*
+ * The stack over n batches held in HOST memory (a library convenience for
+ * streaming callers; the pages have no counterpart): batch i is x_host[i]
+ * ([B, N, D] in dtype, contiguous) and its output goes to y_host[i]. The copy
+ * in of batch i+1 and the copy out of batch i-1 overlap the stack pass of
+ * batch i (two staging slots in `staging`, which the caller owns: size it with
+ * sva_hybrid_stack_host_staging_bytes). Host buffers should be page-locked
+ * for the copies to overlap; pageable memory works but serialises. The call
+ * is asynchronous: it creates two copy streams and a few events and releases
+ * them before returning (the runtime frees them once their work is done);
+ * `stream` runs the stack passes, and once its work up to this call is
+ * complete every y_host[i] holds its result. ws as for sva_hybrid_stack_fwd.
+ */
+size_t sva_hybrid_stack_host_staging_bytes(const sva_stack_desc* desc);
+sva_status_t sva_hybrid_stack_fwd_host(const sva_stack_desc* desc, const void* const* x_host,
+                                       void* const* y_host, int n, void* ws, size_t ws_bytes,
+                                       void* staging, size_t staging_bytes, sva_stream_t stream);
+
 /* Synchronises `stream`, then reads the status word of `ws` (SVA_OK or the
  * first device-side error, e.g. SVA_ERR_DEVICE_TIMEOUT). */
 sva_status_t sva_check_device_status(const void* ws, sva_stream_t stream);

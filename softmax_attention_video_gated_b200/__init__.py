@@ -101,6 +101,11 @@ _SIGS = {
     "sva_hybrid_stack_fwd": (ctypes.c_int, [ctypes.POINTER(StackDesc), ctypes.c_void_p,
                                             ctypes.c_void_p, ctypes.c_void_p, ctypes.c_size_t,
                                             ctypes.c_void_p]),
+    "sva_hybrid_stack_host_staging_bytes": (ctypes.c_size_t, [ctypes.POINTER(StackDesc)]),
+    "sva_hybrid_stack_fwd_host": (ctypes.c_int, [ctypes.POINTER(StackDesc), _c_void_p_p,
+                                                 _c_void_p_p, ctypes.c_int, ctypes.c_void_p,
+                                                 ctypes.c_size_t, ctypes.c_void_p, ctypes.c_size_t,
+                                                 ctypes.c_void_p]),
     "sva_check_device_status": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p]),
     "sva_selftest_bounded_wait": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_size_t, ctypes.c_uint,
                                                  ctypes.c_void_p]),
@@ -371,6 +376,35 @@ def sva_hybrid_stack_fwd(stack: Stack, x, y, ws=None, stream=None):
     _check(_lib().sva_hybrid_stack_fwd(ctypes.byref(stack.desc), _ptr(x), _ptr(y), _ptr(ws),
                                        ws.numel(), _stream(stream)), "sva_hybrid_stack_fwd")
     return ws
+
+
+def sva_hybrid_stack_host_staging_bytes(stack: Stack) -> int:
+    return int(_lib().sva_hybrid_stack_host_staging_bytes(ctypes.byref(stack.desc)))
+
+
+def sva_hybrid_stack_fwd_host(stack: Stack, xs_host: Sequence, ys_host: Sequence, ws=None,
+                              staging=None, stream=None):
+    """The stack over host batches: ys_host[i] = stack(xs_host[i]), copies in and
+    out overlapped with the passes (CPU tensors [B, N, D], contiguous; pin them
+    for the overlap). Asynchronous on `stream`. Returns (ws, staging)."""
+    if len(xs_host) != len(ys_host):
+        raise ValueError("one output per input")
+    for t in list(xs_host) + list(ys_host):
+        if t.is_cuda or not t.is_contiguous():
+            raise ValueError("host batches must be contiguous CPU tensors")
+    torch = _torch()
+    dev = torch.device("cuda", torch.cuda.current_device())
+    ws = workspace(stack.workspace_bytes(), dev) if ws is None else ws
+    if staging is None:
+        staging = workspace(sva_hybrid_stack_host_staging_bytes(stack), dev)
+    n = len(xs_host)
+    xp = (ctypes.c_void_p * max(n, 1))(*[t.data_ptr() for t in xs_host])
+    yp = (ctypes.c_void_p * max(n, 1))(*[t.data_ptr() for t in ys_host])
+    _check(_lib().sva_hybrid_stack_fwd_host(
+        ctypes.byref(stack.desc), ctypes.cast(xp, _c_void_p_p), ctypes.cast(yp, _c_void_p_p), n,
+        _ptr(ws), ws.numel(), _ptr(staging), staging.numel(), _stream(stream)),
+        "sva_hybrid_stack_fwd_host")
+    return ws, staging
 
 
 def sva_check_device_status(ws, stream=None) -> int:

@@ -378,8 +378,12 @@ extern "C" size_t sva_hybrid_stack_workspace_bytes(const sva_stack_desc* desc) {
   return stack_layout(*desc).total;
 }
 
-extern "C" sva_status_t sva_hybrid_stack_fwd(const sva_stack_desc* desc, const void* x, void* y,
-                                             void* ws, size_t ws_bytes, sva_stream_t stream) {
+namespace {
+
+// one stack pass; clear_first resets the workspace status word (a caller
+// running several passes clears it once, so an early device error is kept)
+sva_status_t stack_pass(const sva_stack_desc* desc, const void* x, void* y, void* ws,
+                        size_t ws_bytes, sva_stream_t stream, bool clear_first) {
   sva_status_t st = check_stack(desc);
   if (st != SVA_OK) return st;
   const sva_stack_desc& d = *desc;
@@ -420,7 +424,7 @@ extern "C" sva_status_t sva_hybrid_stack_fwd(const sva_stack_desc* desc, const v
     if ((e = (expr)) != cudaSuccess) return cuda_fail(e); \
   } while (0)
 
-  if ((st = clear_status(ws, s)) != SVA_OK) return st;
+  if (clear_first && (st = clear_status(ws, s)) != SVA_OK) return st;
   {
     ProfScope ps(prof, s, SVA_KERNEL_OTHER);
     SVA_TRY(upcast_to_f32(x, h, rows * D, d.dtype, s));
@@ -526,6 +530,99 @@ extern "C" sva_status_t sva_hybrid_stack_fwd(const sva_stack_desc* desc, const v
   }
 #undef SVA_TRY
   if (d.prof_count != nullptr) *d.prof_count = prof != nullptr ? prof->count : 0;
+  return SVA_OK;
+}
+
+size_t act_slot_bytes(const sva_stack_desc& d) {
+  return align_up(static_cast<size_t>(d.B) * d.N * d.H * d.d * esize(d.dtype), 256);
+}
+
+// streams and events of one host-batch call, released on every exit path
+// (the runtime frees them once the work queued on them is done)
+struct CopyPipe {
+  cudaStream_t h2d = nullptr, d2h = nullptr;
+  cudaEvent_t start = nullptr, in_done[2] = {}, pass_done[2] = {}, out_done[2] = {};
+  ~CopyPipe() {
+    for (cudaEvent_t* e : {&start, &in_done[0], &in_done[1], &pass_done[0], &pass_done[1],
+                           &out_done[0], &out_done[1]})
+      if (*e != nullptr) cudaEventDestroy(*e);
+    if (h2d != nullptr) cudaStreamDestroy(h2d);
+    if (d2h != nullptr) cudaStreamDestroy(d2h);
+  }
+  cudaError_t create() {
+    cudaError_t e = cudaStreamCreateWithFlags(&h2d, cudaStreamNonBlocking);
+    if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&d2h, cudaStreamNonBlocking);
+    for (cudaEvent_t* ev : {&start, &in_done[0], &in_done[1], &pass_done[0], &pass_done[1],
+                            &out_done[0], &out_done[1]})
+      if (e == cudaSuccess) e = cudaEventCreateWithFlags(ev, cudaEventDisableTiming);
+    return e;
+  }
+};
+
+}  // namespace
+
+extern "C" sva_status_t sva_hybrid_stack_fwd(const sva_stack_desc* desc, const void* x, void* y,
+                                             void* ws, size_t ws_bytes, sva_stream_t stream) {
+  return stack_pass(desc, x, y, ws, ws_bytes, stream, true);
+}
+
+extern "C" size_t sva_hybrid_stack_host_staging_bytes(const sva_stack_desc* desc) {
+  if (check_stack(desc) != SVA_OK) return 0;
+  return 4 * act_slot_bytes(*desc);  // two slots, each an input and an output
+}
+
+extern "C" sva_status_t sva_hybrid_stack_fwd_host(const sva_stack_desc* desc,
+                                                  const void* const* x_host, void* const* y_host,
+                                                  int n, void* ws, size_t ws_bytes, void* staging,
+                                                  size_t staging_bytes, sva_stream_t stream) {
+  sva_status_t st = check_stack(desc);
+  if (st != SVA_OK) return st;
+  if (n < 0 || (n > 0 && (x_host == nullptr || y_host == nullptr)))
+    return SVA_ERR_INVALID_ARGUMENT;
+  for (int i = 0; i < n; ++i)
+    if (x_host[i] == nullptr || y_host[i] == nullptr) return SVA_ERR_INVALID_ARGUMENT;
+  const sva_stack_desc& d = *desc;
+  const size_t slot = act_slot_bytes(d);
+  if (staging == nullptr || !aligned16(staging) || staging_bytes < 4 * slot)
+    return SVA_ERR_WORKSPACE;
+  if (ws == nullptr || !aligned16(ws) || ws_bytes < stack_layout(d).total) return SVA_ERR_WORKSPACE;
+  if (n == 0) return SVA_OK;
+  const size_t bytes = static_cast<size_t>(d.B) * d.N * d.H * d.d * esize(d.dtype);
+  char* sb = static_cast<char*>(staging);
+  void* xs[2] = {sb, sb + slot};
+  void* ys[2] = {sb + 2 * slot, sb + 3 * slot};
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  CopyPipe cp;
+  cudaError_t e = cp.create();
+  if (e != cudaSuccess) return cuda_fail(e);
+  if ((st = clear_status(ws, s)) != SVA_OK) return st;
+#define SVA_TRY(expr)                                     \
+  do {                                                    \
+    if ((e = (expr)) != cudaSuccess) return cuda_fail(e); \
+  } while (0)
+  // the copy streams start after the work already queued on `stream`
+  SVA_TRY(cudaEventRecord(cp.start, s));
+  SVA_TRY(cudaStreamWaitEvent(cp.h2d, cp.start, 0));
+  SVA_TRY(cudaStreamWaitEvent(cp.d2h, cp.start, 0));
+  for (int i = 0; i < n; ++i) {
+    const int k = i & 1;
+    // slot k's input is free once the pass of batch i - 2 has finished
+    if (i >= 2) SVA_TRY(cudaStreamWaitEvent(cp.h2d, cp.pass_done[k], 0));
+    SVA_TRY(cudaMemcpyAsync(xs[k], x_host[i], bytes, cudaMemcpyHostToDevice, cp.h2d));
+    SVA_TRY(cudaEventRecord(cp.in_done[k], cp.h2d));
+    // the pass needs its input in and slot k's previous output copied out
+    SVA_TRY(cudaStreamWaitEvent(s, cp.in_done[k], 0));
+    if (i >= 2) SVA_TRY(cudaStreamWaitEvent(s, cp.out_done[k], 0));
+    if ((st = stack_pass(desc, xs[k], ys[k], ws, ws_bytes, stream, false)) != SVA_OK) return st;
+    SVA_TRY(cudaEventRecord(cp.pass_done[k], s));
+    SVA_TRY(cudaStreamWaitEvent(cp.d2h, cp.pass_done[k], 0));
+    SVA_TRY(cudaMemcpyAsync(y_host[i], ys[k], bytes, cudaMemcpyDeviceToHost, cp.d2h));
+    SVA_TRY(cudaEventRecord(cp.out_done[k], cp.d2h));
+  }
+  // `stream` completes only after every output has reached the host
+  SVA_TRY(cudaStreamWaitEvent(s, cp.out_done[(n - 1) & 1], 0));
+  if (n >= 2) SVA_TRY(cudaStreamWaitEvent(s, cp.out_done[n & 1], 0));
+#undef SVA_TRY
   return SVA_OK;
 }
 

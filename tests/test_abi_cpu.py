@@ -120,3 +120,31 @@ def test_stack_workspace_query_and_validation():
     assert rows * 24 * 2 <= n1 - n0 <= rows * 24 * 2 + 2048
     wg[0] = None
     assert lib.sva_hybrid_stack_workspace_bytes(ctypes.byref(d)) == 0
+    d.w_wg = None
+
+
+def test_stack_host_batches_host_validation():
+    # all checks run before any stream, event or copy is made
+    lib = sva._lib()
+    L = 8
+    w = (ctypes.c_void_p * L)(*([0x100000] * L))
+    d = sva.StackDesc()
+    d.B, d.N, d.H, d.d, d.L, d.dtype = 1, 1000, 2, 128, L, sva.SVA_BF16
+    d.softmax_period, d.attnres_block = 4, 8
+    d.w_qkvg = ctypes.cast(w, ctypes.POINTER(ctypes.c_void_p))
+    d.w_o = ctypes.cast(w, ctypes.POINTER(ctypes.c_void_p))
+    d.eps = 1e-6
+    need = lib.sva_hybrid_stack_host_staging_bytes(ctypes.byref(d))
+    assert need >= 4 * 1000 * 256 * 2 and need % 256 == 0
+    ws = lib.sva_hybrid_stack_workspace_bytes(ctypes.byref(d))
+    hx = (ctypes.c_void_p * 2)(0x1000, 0x2000)
+    hy = (ctypes.c_void_p * 2)(0x3000, None)
+    pp = lambda a: ctypes.cast(a, ctypes.POINTER(ctypes.c_void_p))  # noqa: E731
+    call = lambda xs, ys, n, sb: lib.sva_hybrid_stack_fwd_host(  # noqa: E731
+        ctypes.byref(d), xs, ys, n, 0x40000, ws, 0x80000, sb, None)
+    assert call(pp(hx), pp(hy), -1, need) == sva.SVA_ERR_INVALID_ARGUMENT
+    assert call(None, pp(hy), 1, need) == sva.SVA_ERR_INVALID_ARGUMENT
+    assert call(pp(hx), pp(hy), 2, need) == sva.SVA_ERR_INVALID_ARGUMENT   # y_host[1] is NULL
+    assert call(pp(hx), pp(hy), 1, need - 256) == sva.SVA_ERR_WORKSPACE
+    assert lib.sva_hybrid_stack_fwd_host(ctypes.byref(d), pp(hx), pp(hy), 1, 0x40000, ws - 1024,
+                                         0x80000, need, None) == sva.SVA_ERR_WORKSPACE

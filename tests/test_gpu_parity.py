@@ -389,6 +389,26 @@ def test_stack_bf16_zero_write_gate_weights_double_eps():
     assert rel_l2(y_1e - x, y_2e - x) > 2e-2
 
 
+@pytest.mark.parametrize("n", [0, 1, 3])
+def test_stack_host_batches_match_device_passes(n):
+    # the pipelined host-batch call gives, bit for bit, what one device-resident
+    # pass per batch gives (the same kernels on the same inputs)
+    x, wq, wo, wr, H = small_bf16_stack(12, N=300, seed=97)
+    st = sva.Stack([to_dev(w, "bf16") for w in wq], [to_dev(w, "bf16") for w in wo],
+                   to_dev(wr, "bf16"), 1, 300, H)
+    xs = [to_dev(W.round_to(np.random.default_rng(98 + i).standard_normal(x.shape)
+                            .astype(np.float32), "bf16"), "bf16") for i in range(n)]
+    xh = [t.cpu().pin_memory() for t in xs]
+    yh = [torch.empty_like(t).pin_memory() for t in xh]
+    ws, _ = sva.sva_hybrid_stack_fwd_host(st, xh, yh)
+    assert sva.sva_check_device_status(ws) == sva.SVA_OK
+    for i in range(n):
+        y = torch.empty_like(xs[i])
+        sva.sva_hybrid_stack_fwd(st, xs[i], y)
+        torch.cuda.synchronize()
+        assert torch.equal(yh[i], y.cpu()), i
+
+
 def test_stack_bf16_single_block_attnres_on_equals_off():
     x, wq, wo, wr, H = small_bf16_stack(8, N=257, seed=91)
     y_on, _, _ = run_stack(x, wq, wo, wr, H, "bf16", attnres_block=8)

@@ -81,6 +81,8 @@ typedef struct {
   const void* wgate; int64_t ldw;  /* linear attention, nullable [B, N, >=H]:
                                       write-gate logits, one per token and head,
                                       in dtype; row stride ldw >= H elements   */
+  int n_keys;       /* softmax anchor: rows of k and v ([B, n_keys, >=D]) when
+                       the queries are a shard of the sequence; 0 means N     */
 } sva_attn_args;
 
 /*
@@ -105,6 +107,25 @@ sva_status_t sva_linear_attn_fwd(const sva_attn_args* args, void* ws, size_t ws_
                                  sva_stream_t stream);
 
 /*
+ * The two halves of sva_linear_attn_fwd, for callers that shard the tokens
+ * (e.g. across GPUs): the state is a sum over tokens, so the states of the
+ * shards, summed (an all-reduce), are the state of the whole sequence, and
+ * each shard's queries then read it out. The state is fp32, per (batch,
+ * head) d*d + d values: S row-major (row = d_k, column = d_v), then z; size it
+ * with sva_linear_attn_state_bytes (1.58 MB for B = 1, H = 24, d = 128).
+ *   sva_linear_attn_state_fwd:   uses k, v (and wgate) of args->N tokens and
+ *                                writes the state; q, gate, out are ignored.
+ *   sva_linear_attn_readout_fwd: uses q, gate, out (and residual) of args->N
+ *                                query tokens and a given state; k, v ignored.
+ * Workspace as for sva_linear_attn_fwd with the same B, N, H, d, dtype.
+ */
+size_t sva_linear_attn_state_bytes(int B, int H, int d);
+sva_status_t sva_linear_attn_state_fwd(const sva_attn_args* args, float* state, void* ws,
+                                       size_t ws_bytes, sva_stream_t stream);
+sva_status_t sva_linear_attn_readout_fwd(const sva_attn_args* args, const float* state, void* ws,
+                                         size_t ws_bytes, sva_stream_t stream);
+
+/*
  * Allocation-free variant of sva_linear_attn_fwd (same arguments, same
  * results) for callers that cannot allocate device memory when they run the
  * mixer: engines that plan all device memory at start-up and allow no
@@ -125,6 +146,9 @@ sva_status_t sva_linear_attn_fwd_noalloc(const sva_attn_args* args, sva_stream_t
  * [lode.cx summary, "How It Works": gated softmax keeps exact token relations;
  * SANA-Video 2.0 abstract: periodic gated-softmax anchors at a 3:1 ratio]:
  *     Y_t = sum_s softmax_s(scale * Q_t . K_s) V_s  *  sigmoid(G_t)
+ * over the N query rows of q (gate, out, residual) and the n_keys rows of k
+ * and v (n_keys = 0: the same N tokens; otherwise e.g. one shard's queries
+ * against the all-gathered keys and values of the whole sequence).
  * No N x N matrix is stored. Supported: SVA_BF16 with d = 128 (tcgen05 flash
  * kernel), SVA_F32 with d in {64, 128}. Workspace: status word only.
  */

@@ -49,6 +49,7 @@ class AttnArgs(ctypes.Structure):
         ("out", ctypes.c_void_p), ("ldo", ctypes.c_int64),
         ("eps", ctypes.c_float), ("scale", ctypes.c_float), ("flags", ctypes.c_uint),
         ("wgate", ctypes.c_void_p), ("ldw", ctypes.c_int64),
+        ("n_keys", ctypes.c_int),
     ]
 
 
@@ -74,6 +75,13 @@ _SIGS = {
     "sva_linear_attn_fwd": (ctypes.c_int, [ctypes.POINTER(AttnArgs), ctypes.c_void_p,
                                            ctypes.c_size_t, ctypes.c_void_p]),
     "sva_linear_attn_fwd_noalloc": (ctypes.c_int, [ctypes.POINTER(AttnArgs), ctypes.c_void_p]),
+    "sva_linear_attn_state_bytes": (ctypes.c_size_t, [ctypes.c_int] * 3),
+    "sva_linear_attn_state_fwd": (ctypes.c_int, [ctypes.POINTER(AttnArgs), ctypes.c_void_p,
+                                                 ctypes.c_void_p, ctypes.c_size_t,
+                                                 ctypes.c_void_p]),
+    "sva_linear_attn_readout_fwd": (ctypes.c_int, [ctypes.POINTER(AttnArgs), ctypes.c_void_p,
+                                                   ctypes.c_void_p, ctypes.c_size_t,
+                                                   ctypes.c_void_p]),
     "sva_softmax_anchor_workspace_bytes": (ctypes.c_size_t, [ctypes.c_int] * 5),
     "sva_softmax_anchor_fwd": (ctypes.c_int, [ctypes.POINTER(AttnArgs), ctypes.c_void_p,
                                               ctypes.c_size_t, ctypes.c_void_p]),
@@ -192,20 +200,31 @@ def workspace(nbytes: int, device=None):
 
 
 def _attn_args(q, k, v, gate, out, H, residual, eps, scale, flags, wgate=None) -> AttnArgs:
-    B, N, D = q.shape
+    """Marshals an attention call. Operands a call does not use may be None (the
+    linear-attention phases); k and v may hold more rows than q (the anchor over
+    all keys for one shard's queries), which sets n_keys."""
+    lead = q if q is not None else k
+    B, N, D = lead.shape
     if D % H:
         raise ValueError(f"width {D} is not a multiple of H={H}")
-    dt = _dtype_code(q)
-    for t in (k, v, gate, out) + ((residual,) if residual is not None else ()):
-        if _dtype_code(t) != dt:
+    dt = _dtype_code(lead)
+    for t in (q, k, v, gate, out, residual):
+        if t is not None and _dtype_code(t) != dt:
             raise TypeError("q, k, v, gate, out and residual must share one dtype")
     a = AttnArgs()
     a.B, a.N, a.H, a.d, a.dtype = B, N, H, D // H, dt
-    a.q, a.ldq = _ptr(q), _rows(q, B, N)
-    a.k, a.ldk = _ptr(k), _rows(k, B, N)
-    a.v, a.ldv = _ptr(v), _rows(v, B, N)
-    a.gate, a.ldg = _ptr(gate), _rows(gate, B, N)
-    a.out, a.ldo = _ptr(out), _rows(out, B, N)
+    if q is not None:
+        a.q, a.ldq = _ptr(q), _rows(q, B, N)
+    if k is not None:
+        Nk = k.shape[1]
+        a.k, a.ldk = _ptr(k), _rows(k, B, Nk)
+        a.v, a.ldv = _ptr(v), _rows(v, B, Nk)
+        if Nk != N:
+            a.n_keys = Nk
+    if gate is not None:
+        a.gate, a.ldg = _ptr(gate), _rows(gate, B, N)
+    if out is not None:
+        a.out, a.ldo = _ptr(out), _rows(out, B, N)
     if residual is not None:
         a.residual, a.ldr = _ptr(residual), _rows(residual, B, N)
     a.eps, a.scale, a.flags = float(eps), float(scale), int(flags)
@@ -238,6 +257,41 @@ def sva_linear_attn_fwd(q, k, v, gate, out, H: int, residual=None, eps: float = 
     _check(_lib().sva_linear_attn_fwd(ctypes.byref(a), _ptr(ws), ws.numel(), _stream(stream)),
            "sva_linear_attn_fwd")
     return ws
+
+
+def sva_linear_attn_state_bytes(B: int, H: int, d: int) -> int:
+    return int(_lib().sva_linear_attn_state_bytes(B, H, d))
+
+
+def sva_linear_attn_state_fwd(k, v, state, H: int, flags: int = 0, wgate=None, ws=None,
+                              stream=None):
+    """The fp32 state [B*H][d*d + d] (S, then z) of the tokens in k and v."""
+    a = _attn_args(None, k, v, None, None, H, None, 0.0, 0.0, flags, wgate)
+    _check_state(state, a)
+    need = sva_linear_attn_workspace_bytes(a.B, a.N, a.H, a.d, a.dtype)
+    ws = workspace(need, k.device) if ws is None else ws
+    _check(_lib().sva_linear_attn_state_fwd(ctypes.byref(a), _ptr(state), _ptr(ws), ws.numel(),
+                                            _stream(stream)), "sva_linear_attn_state_fwd")
+    return ws
+
+
+def sva_linear_attn_readout_fwd(q, gate, out, state, H: int, residual=None, eps: float = 1e-6,
+                                flags: int = 0, ws=None, stream=None):
+    """Y of the query tokens in q against a given fp32 state (e.g. summed over shards)."""
+    a = _attn_args(q, None, None, gate, out, H, residual, eps, 0.0, flags)
+    _check_state(state, a)
+    need = sva_linear_attn_workspace_bytes(a.B, a.N, a.H, a.d, a.dtype)
+    ws = workspace(need, q.device) if ws is None else ws
+    _check(_lib().sva_linear_attn_readout_fwd(ctypes.byref(a), _ptr(state), _ptr(ws), ws.numel(),
+                                              _stream(stream)), "sva_linear_attn_readout_fwd")
+    return ws
+
+
+def _check_state(state, a):
+    torch = _torch()
+    need = sva_linear_attn_state_bytes(a.B, a.H, a.d) // 4
+    if state.dtype != torch.float32 or not state.is_contiguous() or state.numel() < need:
+        raise ValueError(f"state must be a contiguous fp32 tensor of >= {need} values")
 
 
 def sva_linear_attn_fwd_noalloc(q, k, v, gate, out, H: int, residual=None, eps: float = 1e-6,

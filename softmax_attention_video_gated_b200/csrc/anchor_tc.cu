@@ -117,7 +117,8 @@ __device__ __forceinline__ float ex2_row(float x, int idx) {
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     anchor_tc_kernel(const __grid_constant__ CUtensorMap map_q,
                      const __grid_constant__ CUtensorMap map_k,
-                     const __grid_constant__ CUtensorMap map_v, int N, float scale_log2,
+                     const __grid_constant__ CUtensorMap map_v, int N, int Nk,
+                     float scale_log2,
                      const __nv_bfloat16* gate, int64_t ldg, const __nv_bfloat16* residual,
                      int64_t ldr, __nv_bfloat16* out, int64_t ldo, int* status) {
   extern __shared__ uint8_t smem_raw[];
@@ -127,7 +128,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   const int q0 = blockIdx.x * 2 * BQ, h = blockIdx.y, b = blockIdx.z;
   const int warp = warp_id(), lane = lane_id();
   const int wg = warp >> 2;
-  const int nkv = (N + BKV - 1) / BKV;
+  const int nkv = (Nk + BKV - 1) / BKV;  // key blocks (Nk keys; N query rows)
   const bool has1 = q0 + BQ < N;  // the second tile holds at least one query
 
   if (threadIdx.x == 0) {
@@ -302,7 +303,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         float s[BKV];
 #pragma unroll
         for (int i = 0; i < BKV; ++i) s[i] = __uint_as_float(v[i >> 5][i & 31]);
-        const int valid = N - j * BKV;  // keys of this block inside the sequence
+        const int valid = Nk - j * BKV;  // keys of this block inside the sequence
         if (valid < BKV) {
 #pragma unroll
           for (int i = 0; i < BKV; ++i)
@@ -456,8 +457,9 @@ bool act_map(CUtensorMap* m, const void* base, int64_t ld, int B, int N, int D) 
 cudaError_t anchor_bf16(const sva_attn_args& a, int* status, cudaStream_t s) {
   const int D = a.H * a.d;
   CUtensorMap mq, mk, mv;
-  if (!act_map(&mq, a.q, a.ldq, a.B, a.N, D) || !act_map(&mk, a.k, a.ldk, a.B, a.N, D) ||
-      !act_map(&mv, a.v, a.ldv, a.B, a.N, D))
+  const int Nk = a.n_keys > 0 ? a.n_keys : a.N;
+  if (!act_map(&mq, a.q, a.ldq, a.B, a.N, D) || !act_map(&mk, a.k, a.ldk, a.B, Nk, D) ||
+      !act_map(&mv, a.v, a.ldv, a.B, Nk, D))
     return cudaErrorInvalidValue;
   const float scale = a.scale != 0.f ? a.scale : 1.0f / sqrtf(static_cast<float>(a.d));
   const float scale_log2 = scale * 1.4426950408889634f;
@@ -466,7 +468,7 @@ cudaError_t anchor_bf16(const sva_attn_args& a, int* status, cudaStream_t s) {
   if (e != cudaSuccess) return e;
   dim3 grid((a.N + 2 * BQ - 1) / (2 * BQ), a.H, a.B);
   anchor_tc_kernel<<<grid, NUM_THREADS, kAnchorSmem, s>>>(
-      mq, mk, mv, a.N, scale_log2, static_cast<const __nv_bfloat16*>(a.gate), a.ldg,
+      mq, mk, mv, a.N, Nk, scale_log2, static_cast<const __nv_bfloat16*>(a.gate), a.ldg,
       static_cast<const __nv_bfloat16*>(a.residual), a.ldr, static_cast<__nv_bfloat16*>(a.out),
       a.ldo, status);
   return cudaGetLastError();

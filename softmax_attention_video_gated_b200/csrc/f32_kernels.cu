@@ -209,25 +209,27 @@ __global__ void __launch_bounds__(256) anchor_f32_kernel(sva_attn_args a, float 
   const float* Q = static_cast<const float*>(a.q);
   const float* K = static_cast<const float*>(a.k);
   const float* V = static_cast<const float*>(a.v);
-  const int64_t base = static_cast<int64_t>(b) * a.N;
+  const int64_t base = static_cast<int64_t>(b) * a.N;    // query rows of batch b
+  const int Nk = a.n_keys > 0 ? a.n_keys : a.N;            // keys (all of them)
+  const int64_t kbase = static_cast<int64_t>(b) * Nk;
   for (int i = lane; i < D_; i += 32)
     Qs[w][i] = (t < a.N) ? Q[(base + t) * a.ldq + h * D_ + i] : 0.f;
   float m = -INFINITY, l = 0.f;
   float o[C];
 #pragma unroll
   for (int q = 0; q < C; ++q) o[q] = 0.f;
-  for (int s0 = 0; s0 < a.N; s0 += 32) {
+  for (int s0 = 0; s0 < Nk; s0 += 32) {
     __syncthreads();
     for (int idx = threadIdx.x; idx < 32 * D_; idx += 256) {
       const int r = idx / D_, col = idx % D_;
       const int s = s0 + r;
-      Ks[r][col] = (s < a.N) ? K[(base + s) * a.ldk + h * D_ + col] : 0.f;
-      Vs[r][col] = (s < a.N) ? V[(base + s) * a.ldv + h * D_ + col] : 0.f;
+      Ks[r][col] = (s < Nk) ? K[(kbase + s) * a.ldk + h * D_ + col] : 0.f;
+      Vs[r][col] = (s < Nk) ? V[(kbase + s) * a.ldv + h * D_ + col] : 0.f;
     }
     __syncthreads();
     float sc = 0.f;
     for (int i = 0; i < D_; ++i) sc = fmaf(Qs[w][i], Ks[lane][i], sc);
-    sc = (s0 + lane < a.N) ? sc * scale : -INFINITY;
+    sc = (s0 + lane < Nk) ? sc * scale : -INFINITY;
     float mt = sc;
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, off));
@@ -276,28 +278,34 @@ cudaError_t gemm_f32(const GemmArgs& g, cudaStream_t s) {
 }
 
 cudaError_t linear_f32(const sva_attn_args& a, int* status, void* scratch, cudaStream_t s,
-                       Prof* prof) {
+                       Prof* prof, float* state_out, const float* state_in) {
   (void)status;
   const LinearPlan p = linear_plan(a.B, a.N, a.H, a.d, SVA_F32);
   char* base = static_cast<char*>(scratch);
   float* partial = reinterpret_cast<float*>(base + p.partial_off);
-  float* state = reinterpret_cast<float*>(base + p.state_off);
+  const float* state = state_in;
   const int elems = a.d * a.d + a.d;
-  {
-    ProfScope ps(prof, s, SVA_KERNEL_LINEAR_STATE);
-    dim3 grid(p.n_chunks, a.H, a.B);
-    if (a.d == 64)
-      lin_state_f32_kernel<64><<<grid, 256, 0, s>>>(a, partial, p.tiles_per_chunk, p.n_chunks);
-    else
-      lin_state_f32_kernel<128><<<grid, 256, 0, s>>>(a, partial, p.tiles_per_chunk, p.n_chunks);
-    cudaError_t e = cudaGetLastError();
-    if (e != cudaSuccess) return e;
-  }
-  {
-    ProfScope ps(prof, s, SVA_KERNEL_LINEAR_REDUCE);
-    lin_reduce_f32_kernel<<<a.B * a.H, 256, 0, s>>>(partial, state, p.n_chunks, elems);
-    cudaError_t e = cudaGetLastError();
-    if (e != cudaSuccess) return e;
+  if (state_in == nullptr) {
+    {
+      ProfScope ps(prof, s, SVA_KERNEL_LINEAR_STATE);
+      dim3 grid(p.n_chunks, a.H, a.B);
+      if (a.d == 64)
+        lin_state_f32_kernel<64><<<grid, 256, 0, s>>>(a, partial, p.tiles_per_chunk, p.n_chunks);
+      else
+        lin_state_f32_kernel<128><<<grid, 256, 0, s>>>(a, partial, p.tiles_per_chunk, p.n_chunks);
+      cudaError_t e = cudaGetLastError();
+      if (e != cudaSuccess) return e;
+    }
+    // the state goes to the caller (state only) or to the scratch (fused)
+    float* dst = state_out != nullptr ? state_out : reinterpret_cast<float*>(base + p.state_off);
+    {
+      ProfScope ps(prof, s, SVA_KERNEL_LINEAR_REDUCE);
+      lin_reduce_f32_kernel<<<a.B * a.H, 256, 0, s>>>(partial, dst, p.n_chunks, elems);
+      cudaError_t e = cudaGetLastError();
+      if (e != cudaSuccess) return e;
+    }
+    if (state_out != nullptr) return cudaSuccess;
+    state = dst;
   }
   ProfScope ps(prof, s, SVA_KERNEL_LINEAR_READOUT);
   dim3 grid((a.N + LT - 1) / LT, a.H, a.B);

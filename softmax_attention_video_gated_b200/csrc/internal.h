@@ -82,10 +82,14 @@ struct LinearPlan {
   size_t partial_off = 0, state_off = 0, total = 0;
 };
 LinearPlan linear_plan(int B, int N, int H, int d, sva_dtype_t dt);
+// Gated linear attention. With state_out, only the state pass runs and the
+// fp32 state [B*H][d*d + d] (S row-major d_k x d_v, then z) is written there;
+// with state_in, the state pass is skipped and the read-out uses that state;
+// with neither, the fused layer.
 cudaError_t linear_bf16(const sva_attn_args& a, int* status, void* scratch, cudaStream_t s,
-                        Prof* prof);
+                        Prof* prof, float* state_out = nullptr, const float* state_in = nullptr);
 cudaError_t linear_f32(const sva_attn_args& a, int* status, void* scratch, cudaStream_t s,
-                       Prof* prof);
+                       Prof* prof, float* state_out = nullptr, const float* state_in = nullptr);
 
 // ---------------------------------------------------------------- softmax anchor
 cudaError_t anchor_bf16(const sva_attn_args& a, int* status, cudaStream_t s);

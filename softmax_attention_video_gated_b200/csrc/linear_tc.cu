@@ -343,6 +343,21 @@ __global__ void __launch_bounds__(256) lin_reduce_bf16_kernel(const float* __res
   }
 }
 
+// fp32 state of one (batch, head), [S (d_k rows x d_v) | z]: the chunk partials
+// summed in chunk order (the same order as the fused path's reduce)
+__global__ void __launch_bounds__(256) lin_sum_chunks_kernel(const float* __restrict__ partial,
+                                                             float* __restrict__ state,
+                                                             int n_chunks) {
+  const int elems = HD * HD + HD;
+  const int64_t bh = blockIdx.y;
+  const int e = blockIdx.x * 256 + threadIdx.x;
+  if (e >= elems) return;
+  const float* p = partial + bh * n_chunks * elems + e;
+  float acc = 0.f;
+  for (int c = 0; c < n_chunks; ++c) acc += p[static_cast<int64_t>(c) * elems];
+  state[bh * elems + e] = acc;
+}
+
 // ------------------------------------------------------------------ read-out
 // Persistent over the state pass's chunks (one CTA per (token chunk, head,
 // batch), one wave). The head's read-out operand [S^T | z_hi | z_lo | 0] is
@@ -646,15 +661,49 @@ LinearPlan linear_plan(int B, int N, int H, int d, sva_dtype_t dt) {
 }
 
 cudaError_t linear_bf16(const sva_attn_args& a, int* status, void* scratch, cudaStream_t s,
-                        Prof* prof) {
+                        Prof* prof, float* state_out, const float* state_in) {
   const LinearPlan p = linear_plan(a.B, a.N, a.H, a.d, SVA_BF16);
   char* base = static_cast<char*>(scratch);
   float* partial = reinterpret_cast<float*>(base + p.partial_off);
   __nv_bfloat16* state = reinterpret_cast<__nv_bfloat16*>(base + p.state_off);
   const int D = a.H * a.d;
-  CUtensorMap mk, mv, mq, mg, mo, ms;
-  if (!act_map(&mk, a.k, a.ldk, a.B, a.N, D) || !act_map(&mv, a.v, a.ldv, a.B, a.N, D) ||
-      !act_map(&mq, a.q, a.ldq, a.B, a.N, D) || !act_map(&mg, a.gate, a.ldg, a.B, a.N, D))
+  cudaError_t e;
+  if (state_in == nullptr) {
+    // ------------------------------------------------ state pass (K, V of these tokens)
+    CUtensorMap mk, mv;
+    if (!act_map(&mk, a.k, a.ldk, a.B, a.N, D) || !act_map(&mv, a.v, a.ldv, a.B, a.N, D))
+      return cudaErrorInvalidValue;
+    {
+      ProfScope ps(prof, s, SVA_KERNEL_LINEAR_STATE);
+      const bool wg = a.wgate != nullptr;
+      auto kern = wg ? lin_state_tc_kernel<true> : lin_state_tc_kernel<false>;
+      e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               static_cast<int>(kStateSmem));
+      if (e != cudaSuccess) return e;
+      dim3 grid(p.n_chunks, a.H, a.B);
+      kern<<<grid, 192, kStateSmem, s>>>(mk, mv, a.N, a.H, p.tiles_per_chunk, p.n_chunks,
+                                         a.flags, static_cast<const __nv_bfloat16*>(a.wgate),
+                                         a.ldw, partial, status);
+      if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    }
+    ProfScope ps(prof, s, SVA_KERNEL_LINEAR_REDUCE);
+    if (state_out != nullptr) {
+      // state only: the fp32 state, for the caller to sum over token shards
+      lin_sum_chunks_kernel<<<dim3((HD * HD + HD + 255) / 256, a.B * a.H), 256, 0, s>>>(
+          partial, state_out, p.n_chunks);
+      return cudaGetLastError();
+    }
+    lin_reduce_bf16_kernel<<<dim3(16, a.B * a.H), 256, 0, s>>>(partial, state, p.n_chunks);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  } else {
+    // read-out of a given fp32 state: its read-out operand, as from one chunk
+    ProfScope ps(prof, s, SVA_KERNEL_LINEAR_REDUCE);
+    lin_reduce_bf16_kernel<<<dim3(16, a.B * a.H), 256, 0, s>>>(state_in, state, 1);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  }
+  // ------------------------------------------------ read-out (Q, G, Y of these tokens)
+  CUtensorMap mq, mg, mo, ms;
+  if (!act_map(&mq, a.q, a.ldq, a.B, a.N, D) || !act_map(&mg, a.gate, a.ldg, a.B, a.N, D))
     return cudaErrorInvalidValue;
   {
     // Y: one [64 x 32] box per epilogue warp
@@ -674,25 +723,6 @@ cudaError_t linear_bf16(const sva_attn_args& a, int* status, void* scratch, cuda
     if (!encode_tmap(&ms, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, state, dims, strides, box,
                      CU_TENSOR_MAP_SWIZZLE_128B))
       return cudaErrorInvalidValue;
-  }
-  cudaError_t e;
-  {
-    ProfScope ps(prof, s, SVA_KERNEL_LINEAR_STATE);
-    const bool wg = a.wgate != nullptr;
-    auto kern = wg ? lin_state_tc_kernel<true> : lin_state_tc_kernel<false>;
-    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(kStateSmem));
-    if (e != cudaSuccess) return e;
-    dim3 grid(p.n_chunks, a.H, a.B);
-    kern<<<grid, 192, kStateSmem, s>>>(mk, mv, a.N, a.H, p.tiles_per_chunk, p.n_chunks, a.flags,
-                                       static_cast<const __nv_bfloat16*>(a.wgate), a.ldw,
-                                       partial, status);
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  }
-  {
-    ProfScope ps(prof, s, SVA_KERNEL_LINEAR_REDUCE);
-    lin_reduce_bf16_kernel<<<dim3(16, a.B * a.H), 256, 0, s>>>(partial, state, p.n_chunks);
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
   ProfScope ps(prof, s, SVA_KERNEL_LINEAR_READOUT);
   e = cudaFuncSetAttribute(lin_readout_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,

@@ -77,6 +77,7 @@ extern "C" sva_status_t sva_linear_attn_fwd_noalloc(const sva_attn_args* a, sva_
   if (a->residual != nullptr && (!ptr_ok(a->residual) || !row_ok(a->ldr, D, es)))
     return SVA_ERR_INVALID_ARGUMENT;
   if (!(a->eps >= 0.f && std::isfinite(a->eps))) return SVA_ERR_INVALID_ARGUMENT;
+  if (a->n_keys != 0) return SVA_ERR_INVALID_ARGUMENT;  // a key count is for anchors only
   if (a->wgate != nullptr &&
       (a->ldw < a->H || reinterpret_cast<uintptr_t>(a->wgate) % es != 0))
     return SVA_ERR_INVALID_ARGUMENT;

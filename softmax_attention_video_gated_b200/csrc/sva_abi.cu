@@ -93,22 +93,28 @@ using namespace sva;
 
 namespace {
 
-sva_status_t check_attn(const sva_attn_args* a, bool linear) {
+// need_kv: k, v (and the write gate) are read; need_qgo: q, gate, out (and the
+// residual) are used. The fused calls need both; the two linear-attention
+// phases one each.
+sva_status_t check_attn(const sva_attn_args* a, bool linear, bool need_kv = true,
+                        bool need_qgo = true) {
   if (a == nullptr) return SVA_ERR_INVALID_ARGUMENT;
   if (a->dtype != SVA_F32 && a->dtype != SVA_BF16) return SVA_ERR_INVALID_ARGUMENT;
   if (a->B < 1 || a->N < 1 || a->H < 1 || a->d < 1) return SVA_ERR_INVALID_ARGUMENT;
-  if (a->q == nullptr || a->k == nullptr || a->v == nullptr || a->gate == nullptr ||
-      a->out == nullptr)
-    return SVA_ERR_INVALID_ARGUMENT;
   const int64_t D = static_cast<int64_t>(a->H) * a->d;
-  const void* ptrs[6] = {a->q, a->k, a->v, a->gate, a->out, a->residual};
-  const int64_t lds[6] = {a->ldq, a->ldk, a->ldv, a->ldg, a->ldo, a->ldr};
+  const void* ptrs[6] = {a->k, a->v, a->q, a->gate, a->out, a->residual};
+  const int64_t lds[6] = {a->ldk, a->ldv, a->ldq, a->ldg, a->ldo, a->ldr};
   for (int i = 0; i < 6; ++i) {
+    if (i < 2 && !need_kv) continue;
+    if (i >= 2 && !need_qgo) break;
     if (i == 5 && a->residual == nullptr) break;
-    if (!aligned16(ptrs[i]) || !ld_ok(lds[i], D, a->dtype)) return SVA_ERR_INVALID_ARGUMENT;
+    if (ptrs[i] == nullptr || !aligned16(ptrs[i]) || !ld_ok(lds[i], D, a->dtype))
+      return SVA_ERR_INVALID_ARGUMENT;
   }
   if (linear && !(a->eps >= 0.f && std::isfinite(a->eps))) return SVA_ERR_INVALID_ARGUMENT;
-  if (linear && a->wgate != nullptr &&
+  if (a->n_keys < 0 || (linear && a->n_keys != 0)) return SVA_ERR_INVALID_ARGUMENT;
+  if (static_cast<int64_t>(a->B) * a->n_keys > (int64_t(1) << 31)) return SVA_ERR_UNSUPPORTED;
+  if (linear && need_kv && a->wgate != nullptr &&
       (a->ldw < a->H || reinterpret_cast<uintptr_t>(a->wgate) % esize(a->dtype) != 0))
     return SVA_ERR_INVALID_ARGUMENT;
   if (!linear && !(std::isfinite(a->scale) && a->scale >= 0.f)) return SVA_ERR_INVALID_ARGUMENT;
@@ -159,6 +165,49 @@ extern "C" sva_status_t sva_linear_attn_fwd(const sva_attn_args* args, void* ws,
   void* scratch = static_cast<char*>(ws) + SVA_STATUS_BYTES;
   cudaError_t e = args->dtype == SVA_BF16 ? linear_bf16(*args, status, scratch, s, nullptr)
                                           : linear_f32(*args, status, scratch, s, nullptr);
+  return e == cudaSuccess ? SVA_OK : cuda_fail(e);
+}
+
+extern "C" size_t sva_linear_attn_state_bytes(int B, int H, int d) {
+  if (B < 1 || H < 1 || d < 1) return 0;
+  return static_cast<size_t>(B) * H * (static_cast<size_t>(d) * d + d) * sizeof(float);
+}
+
+extern "C" sva_status_t sva_linear_attn_state_fwd(const sva_attn_args* args, float* state,
+                                                  void* ws, size_t ws_bytes,
+                                                  sva_stream_t stream) {
+  sva_status_t st = check_attn(args, true, true, false);
+  if (st != SVA_OK) return st;
+  if (state == nullptr || !aligned16(state)) return SVA_ERR_INVALID_ARGUMENT;
+  if (ws == nullptr || !aligned16(ws) ||
+      ws_bytes < sva_linear_attn_workspace_bytes(args->B, args->N, args->H, args->d, args->dtype))
+    return SVA_ERR_WORKSPACE;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if ((st = clear_status(ws, s)) != SVA_OK) return st;
+  int* status = static_cast<int*>(ws);
+  void* scratch = static_cast<char*>(ws) + SVA_STATUS_BYTES;
+  const cudaError_t e = args->dtype == SVA_BF16
+                            ? linear_bf16(*args, status, scratch, s, nullptr, state, nullptr)
+                            : linear_f32(*args, status, scratch, s, nullptr, state, nullptr);
+  return e == cudaSuccess ? SVA_OK : cuda_fail(e);
+}
+
+extern "C" sva_status_t sva_linear_attn_readout_fwd(const sva_attn_args* args, const float* state,
+                                                    void* ws, size_t ws_bytes,
+                                                    sva_stream_t stream) {
+  sva_status_t st = check_attn(args, true, false, true);
+  if (st != SVA_OK) return st;
+  if (state == nullptr || !aligned16(state)) return SVA_ERR_INVALID_ARGUMENT;
+  if (ws == nullptr || !aligned16(ws) ||
+      ws_bytes < sva_linear_attn_workspace_bytes(args->B, args->N, args->H, args->d, args->dtype))
+    return SVA_ERR_WORKSPACE;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if ((st = clear_status(ws, s)) != SVA_OK) return st;
+  int* status = static_cast<int*>(ws);
+  void* scratch = static_cast<char*>(ws) + SVA_STATUS_BYTES;
+  const cudaError_t e = args->dtype == SVA_BF16
+                            ? linear_bf16(*args, status, scratch, s, nullptr, nullptr, state)
+                            : linear_f32(*args, status, scratch, s, nullptr, nullptr, state);
   return e == cudaSuccess ? SVA_OK : cuda_fail(e);
 }
 

@@ -57,6 +57,7 @@ def _args(**kw):
     (dict(dtype=7), sva.SVA_ERR_INVALID_ARGUMENT),
     (dict(wgate=0x30000, ldw=1), sva.SVA_ERR_INVALID_ARGUMENT),  # write gate: ldw < H
     (dict(wgate=0x30001, ldw=8), sva.SVA_ERR_INVALID_ARGUMENT),  # not element-aligned
+    (dict(n_keys=500), sva.SVA_ERR_INVALID_ARGUMENT),           # keys count: anchors only
 ])
 def test_linear_attn_rejects_bad_arguments_on_host(bad, expect):
     a = _args(**bad)
@@ -64,6 +65,28 @@ def test_linear_attn_rejects_bad_arguments_on_host(bad, expect):
     assert st == expect
     # the allocation-free entry point validates the same way
     assert sva._lib().sva_linear_attn_fwd_noalloc(ctypes.byref(a), None) == expect
+
+
+def test_phase_and_key_count_host_validation():
+    lib = sva._lib()
+    st = 0x50000
+    # the state phase needs k and v but not q, gate, out; the read-out the reverse
+    a = _args(q=None, gate=None, out=None)
+    assert lib.sva_linear_attn_state_fwd(ctypes.byref(a), None, 0x20000, 1 << 30,
+                                         None) == sva.SVA_ERR_INVALID_ARGUMENT   # no state
+    a = _args(k=None)
+    assert lib.sva_linear_attn_state_fwd(ctypes.byref(a), st, 0x20000, 1 << 30,
+                                         None) == sva.SVA_ERR_INVALID_ARGUMENT
+    a = _args(out=None)
+    assert lib.sva_linear_attn_readout_fwd(ctypes.byref(a), st, 0x20000, 1 << 30,
+                                           None) == sva.SVA_ERR_INVALID_ARGUMENT
+    a = _args(k=None, v=None)
+    assert lib.sva_linear_attn_readout_fwd(ctypes.byref(a), st, 0x20000, 16,
+                                           None) == sva.SVA_ERR_WORKSPACE    # k, v not needed
+    assert lib.sva_linear_attn_state_bytes(1, 24, 128) == 24 * (128 * 128 + 128) * 4
+    a = _args(n_keys=-1)
+    assert lib.sva_softmax_anchor_fwd(ctypes.byref(a), 0x20000, 256,
+                                      None) == sva.SVA_ERR_INVALID_ARGUMENT
 
 
 def test_workspace_checks_happen_before_launch():

@@ -193,6 +193,57 @@ def test_write_gated_linear_attn_noalloc_matches_workspace_call():
     assert torch.equal(out1, out2)
 
 
+# ------------------------------------------------------------------ sequence-sharded cores
+
+@pytest.mark.parametrize("dtype,d", [("bf16", 128), ("f32", 64)])
+@pytest.mark.parametrize("gated", [False, True])
+def test_linear_state_and_readout_phases_over_two_shards(dtype, d, gated):
+    # the states of two token shards, summed (what an all-reduce over two ranks
+    # gives), read out by each shard's queries: the unsharded layer
+    B, N, H = 2, 1000, 2
+    x, t = core_case(B, N, H, d, dtype, seed=51 + d)
+    wg, twg = wgate_case(B, N, H, dtype, 52, 8) if gated else (None, None)
+    cut = 433
+    st = [torch.empty(sva.sva_linear_attn_state_bytes(B, H, d) // 4, device="cuda") for _ in range(2)]
+    outs = []
+    for i, (a, b) in enumerate(((0, cut), (cut, N))):
+        sl = lambda z: z[:, a:b].contiguous()  # noqa: E731
+        sva.sva_linear_attn_state_fwd(sl(t["k"]), sl(t["v"]), st[i], H,
+                                      wgate=None if twg is None else sl(twg))
+    total = st[0] + st[1]
+    for a, b in ((0, cut), (cut, N)):
+        sl = lambda z: z[:, a:b].contiguous()  # noqa: E731
+        o = torch.empty_like(sl(t["q"]))
+        ws = sva.sva_linear_attn_readout_fwd(sl(t["q"]), sl(t["g"]), o, total, H, eps=1e-6)
+        assert sva.sva_check_device_status(ws) == sva.SVA_OK
+        outs.append(o)
+    got = to_host(torch.cat(outs, dim=1))
+    ref = O.linear_attn(x["q"], x["k"], x["v"], x["g"], H, eps=1e-6, wgate=wg)
+    assert_close(got, ref, dtype, "linear phases over two shards")
+    # and the fp32 state itself against the oracle's S and z
+    S, z = O.lin_state(x["k"], x["v"], H, wg)
+    flat = np.concatenate([S.reshape(B * H, -1), z.reshape(B * H, -1)], axis=1).reshape(-1)
+    assert rel_l2(to_host(total), flat) < (1e-2 if dtype == "bf16" else 1e-5)
+
+
+@pytest.mark.parametrize("dtype,d", [("bf16", 128), ("f32", 64), ("f32", 128)])
+@pytest.mark.parametrize("rows,keys", [((300, 777), 1000), ((0, 1000), 300), ((999, 1000), 1000)])
+def test_softmax_anchor_query_shard_against_all_keys(dtype, d, rows, keys):
+    # a shard's queries against the keys and values of the whole sequence
+    # (n_keys != N), including more queries than keys and a one-row shard
+    B, H = 2, 2
+    a, b = rows
+    nq = max(b, keys)
+    x, t = core_case(B, nq, H, d, dtype, seed=61 + a + keys)
+    q, g = t["q"][:, a:b].contiguous(), t["g"][:, a:b].contiguous()
+    k, v = t["k"][:, :keys].contiguous(), t["v"][:, :keys].contiguous()
+    out = torch.empty_like(q)
+    ws = sva.sva_softmax_anchor_fwd(q, k, v, g, out, H)
+    assert sva.sva_check_device_status(ws) == sva.SVA_OK
+    ref = O.softmax_anchor(x["q"][:, a:b], x["k"][:, :keys], x["v"][:, :keys], x["g"][:, a:b], H)
+    assert_close(to_host(out), ref, dtype, f"anchor rows {a}:{b} keys {keys}")
+
+
 # ------------------------------------------------------------------ gated softmax anchor
 
 @pytest.mark.parametrize("dtype,d", [("bf16", 128), ("f32", 64), ("f32", 128)])

@@ -429,7 +429,7 @@ def run_case(args):
                       for tag in (W.TAG_Q, W.TAG_K, W.TAG_V, W.TAG_G))
         out = torch.empty_like(q)
         if args.case == "anchor":
-            ws = sva.workspace(256)
+            ws = sva.workspace(sva._lib().sva_softmax_anchor_workspace_bytes(B, N, H, d, sva.SVA_BF16))
             fn = lambda: sva.sva_softmax_anchor_fwd(q, k, v, g, out, H, ws=ws)  # noqa: E731
             work, unit = 4.0 * B * N * N * D, "TFLOP/s"
         else:

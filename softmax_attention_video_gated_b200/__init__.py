@@ -308,7 +308,8 @@ def sva_softmax_anchor_fwd(q, k, v, gate, out, H: int, residual=None, scale: flo
                            ws=None, stream=None):
     """Gated softmax anchor: out = softmax(scale Q K^T) V * sigmoid(G) (+ residual)."""
     a = _attn_args(q, k, v, gate, out, H, residual, 0.0, scale, 0)
-    ws = workspace(SVA_STATUS_BYTES, q.device) if ws is None else ws
+    need = int(_lib().sva_softmax_anchor_workspace_bytes(a.B, a.N, a.H, a.d, a.dtype))
+    ws = workspace(need, q.device) if ws is None else ws
     _check(_lib().sva_softmax_anchor_fwd(ctypes.byref(a), _ptr(ws), ws.numel(), _stream(stream)),
            "sva_softmax_anchor_fwd")
     return ws

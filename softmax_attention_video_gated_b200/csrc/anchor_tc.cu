@@ -114,21 +114,46 @@ __device__ __forceinline__ float ex2_row(float x, int idx) {
   return ex2_mufu(x);
 }
 
+// Work of one launch: units (query-tile pair, head, batch), x fastest. The
+// first n_full units run whole, one CTA each. The remaining units (the last,
+// partial wave) are split `split` ways along the key blocks. Each part writes
+// its unnormalised O, running max m and row sum l to `partial` and
+// anchor_merge_kernel combines them. This shortens a last wave that would leave
+// most SMs idle. 720p (1,824 units, 48 in the last wave, split 3): the span
+// of the kernel drops from 3.95 to 3.85 ms on one B200, and launch to launch
+// (merge included, 14 us) from 3.96-4.01 to 3.95-3.99 ms. It pays most when
+// a call has fewer units than SMs.
+struct AnchorWork {
+  int n_qpairs, H, n_full, n_split_units, split, nkv_total;
+  float* partial;  // [n_split_units][split][2 tiles][BQ x HD O | BQ x (m, l)]
+};
+constexpr int PART_FLOATS = BQ * HD + 2 * BQ;
+
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     anchor_tc_kernel(const __grid_constant__ CUtensorMap map_q,
                      const __grid_constant__ CUtensorMap map_k,
                      const __grid_constant__ CUtensorMap map_v, int N, int Nk,
-                     float scale_log2,
+                     float scale_log2, AnchorWork wk,
                      const __nv_bfloat16* gate, int64_t ldg, const __nv_bfloat16* residual,
                      int64_t ldr, __nv_bfloat16* out, int64_t ldo, int* status) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
   AnchorTail* tl = reinterpret_cast<AnchorTail*>(smem + TAIL_OFF);
-  const int q0 = blockIdx.x * 2 * BQ, h = blockIdx.y, b = blockIdx.z;
+  // this CTA's unit and key blocks [kb0, kb0 + nkv)
+  int unit = blockIdx.x, kb0 = 0, nkv = wk.nkv_total, part = -1, su = 0;
+  if (unit >= wk.n_full) {
+    const int sidx = unit - wk.n_full;
+    su = sidx / wk.split;
+    part = sidx - su * wk.split;
+    unit = wk.n_full + su;
+    kb0 = part * wk.nkv_total / wk.split;
+    nkv = (part + 1) * wk.nkv_total / wk.split - kb0;
+  }
+  const int q0 = (unit % wk.n_qpairs) * 2 * BQ;
+  const int h = (unit / wk.n_qpairs) % wk.H, b = unit / (wk.n_qpairs * wk.H);
   const int warp = warp_id(), lane = lane_id();
   const int wg = warp >> 2;
-  const int nkv = (Nk + BKV - 1) / BKV;  // key blocks (Nk keys; N query rows)
   const bool has1 = q0 + BQ < N;  // the second tile holds at least one query
 
   if (threadIdx.x == 0) {
@@ -187,8 +212,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         }
         uint8_t* kt = smem + K_OFF + st * 2 * BOX;
         mbar_arrive_expect_tx(&tl->k_full[st], 2 * BOX);
-        tma_load_3d(&map_k, &tl->k_full[st], kt, h * HD, j * BKV, b);
-        tma_load_3d(&map_k, &tl->k_full[st], kt + BOX, h * HD + 64, j * BKV, b);
+        tma_load_3d(&map_k, &tl->k_full[st], kt, h * HD, (kb0 + j) * BKV, b);
+        tma_load_3d(&map_k, &tl->k_full[st], kt + BOX, h * HD + 64, (kb0 + j) * BKV, b);
         ++issued;
       }
       (void)drain_wait(&tl->q_full, 0);
@@ -208,8 +233,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         }
         uint8_t* vt = smem + V_OFF + st * 2 * BOX;
         mbar_arrive_expect_tx(&tl->v_full[st], 2 * BOX);
-        tma_load_3d(&map_v, &tl->v_full[st], vt, h * HD, j * BKV, b);
-        tma_load_3d(&map_v, &tl->v_full[st], vt + BOX, h * HD + 64, j * BKV, b);
+        tma_load_3d(&map_v, &tl->v_full[st], vt, h * HD, (kb0 + j) * BKV, b);
+        tma_load_3d(&map_v, &tl->v_full[st], vt + BOX, h * HD + 64, (kb0 + j) * BKV, b);
         ++issued;
       }
       if (!ok)
@@ -303,7 +328,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         float s[BKV];
 #pragma unroll
         for (int i = 0; i < BKV; ++i) s[i] = __uint_as_float(v[i >> 5][i & 31]);
-        const int valid = Nk - j * BKV;  // keys of this block inside the sequence
+        const int valid = Nk - (kb0 + j) * BKV;  // keys of this block inside the sequence
         if (valid < BKV) {
 #pragma unroll
           for (int i = 0; i < BKV; ++i)
@@ -390,7 +415,23 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         bool w = mbar_wait(&tl->o_done, 0, abort_flag, status, WHERE_ANCHOR);
         ok = __all_sync(0xffffffffu, w);
       }
-      if (ok) {
+      if (ok && part >= 0) {
+        // one part of a split unit: unnormalised O, m and l for the merge
+        tc_fence_after();
+        float* pb = wk.partial + (static_cast<int64_t>(su * wk.split + part) * 2 + t) * PART_FLOATS;
+#pragma unroll 1
+        for (int c = 0; c < HD; c += 32) {
+          uint32_t o[32];
+          tmem_ld32(o_col + c, o);
+          tmem_wait_ld();
+          float4* dst = reinterpret_cast<float4*>(pb + r * HD + c);
+#pragma unroll
+          for (int k = 0; k < 8; ++k)
+            dst[k] = make_float4(__uint_as_float(o[4 * k]), __uint_as_float(o[4 * k + 1]),
+                                 __uint_as_float(o[4 * k + 2]), __uint_as_float(o[4 * k + 3]));
+        }
+        *reinterpret_cast<float2*>(pb + BQ * HD + 2 * r) = make_float2(m, l);
+      } else if (ok) {
         tc_fence_after();
         const int row_t = q0 + t * BQ + r;
         const float inv = 1.0f / l;
@@ -442,6 +483,60 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   }
 }
 
+// Combines the parts of the split units: with M = max_p m_p and w_p =
+// 2^(m_p - M), O = sum_p w_p O_p and l = sum_p w_p l_p (each part's O and l
+// are relative to its own running max), then Y = O / l * sigmoid(G)
+// (+ residual). One warp per query row, four columns per lane.
+__global__ void __launch_bounds__(256) anchor_merge_kernel(AnchorWork wk, int N,
+                                                           const __nv_bfloat16* gate, int64_t ldg,
+                                                           const __nv_bfloat16* residual,
+                                                           int64_t ldr, __nv_bfloat16* out,
+                                                           int64_t ldo) {
+  const int64_t wid = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  if (wid >= static_cast<int64_t>(wk.n_split_units) * 2 * BQ) return;
+  const int su = static_cast<int>(wid / (2 * BQ));
+  const int t = static_cast<int>((wid / BQ) & 1), r = static_cast<int>(wid % BQ);
+  const int unit = wk.n_full + su;
+  const int q0 = (unit % wk.n_qpairs) * 2 * BQ;
+  const int h = (unit / wk.n_qpairs) % wk.H, b = unit / (wk.n_qpairs * wk.H);
+  const int row_t = q0 + t * BQ + r;
+  if (row_t >= N) return;
+  float mx = -INFINITY;
+  for (int p = 0; p < wk.split; ++p) {
+    const float* pb = wk.partial + (static_cast<int64_t>(su * wk.split + p) * 2 + t) * PART_FLOATS;
+    mx = fmaxf(mx, pb[BQ * HD + 2 * r]);
+  }
+  float acc[4] = {0.f, 0.f, 0.f, 0.f}, l = 0.f;
+  for (int p = 0; p < wk.split; ++p) {
+    const float* pb = wk.partial + (static_cast<int64_t>(su * wk.split + p) * 2 + t) * PART_FLOATS;
+    const float2 ml = *reinterpret_cast<const float2*>(pb + BQ * HD + 2 * r);
+    const float w = ml.x == -INFINITY ? 0.f : exp2f(ml.x - mx);
+    const float4 o = *reinterpret_cast<const float4*>(pb + r * HD + 4 * lane);
+    acc[0] = fmaf(w, o.x, acc[0]);
+    acc[1] = fmaf(w, o.y, acc[1]);
+    acc[2] = fmaf(w, o.z, acc[2]);
+    acc[3] = fmaf(w, o.w, acc[3]);
+    l = fmaf(w, ml.y, l);
+  }
+  const float inv = 1.0f / l;
+  const int64_t row = static_cast<int64_t>(b) * N + row_t;
+  const int col = h * HD + 4 * lane;
+  const uint2 gv = *reinterpret_cast<const uint2*>(gate + row * ldg + col);
+  const float gg[4] = {bf16lo_to_f32(gv.x), bf16hi_to_f32(gv.x), bf16lo_to_f32(gv.y),
+                       bf16hi_to_f32(gv.y)};
+  float y[4];
+#pragma unroll
+  for (int e = 0; e < 4; ++e) y[e] = acc[e] * inv * fast_sigmoid(gg[e]);
+  if (residual != nullptr) {
+    const uint2 rv = *reinterpret_cast<const uint2*>(residual + row * ldr + col);
+    y[0] += bf16lo_to_f32(rv.x); y[1] += bf16hi_to_f32(rv.x);
+    y[2] += bf16lo_to_f32(rv.y); y[3] += bf16hi_to_f32(rv.y);
+  }
+  *reinterpret_cast<uint2*>(out + row * ldo + col) =
+      make_uint2(pack_bf16x2(y[0], y[1]), pack_bf16x2(y[2], y[3]));
+}
+
 bool act_map(CUtensorMap* m, const void* base, int64_t ld, int B, int N, int D) {
   const uint64_t dims[3] = {static_cast<uint64_t>(D), static_cast<uint64_t>(N),
                             static_cast<uint64_t>(B)};
@@ -454,23 +549,68 @@ bool act_map(CUtensorMap* m, const void* base, int64_t ld, int B, int N, int D) 
 
 }  // namespace
 
-cudaError_t anchor_bf16(const sva_attn_args& a, int* status, cudaStream_t s) {
+AnchorPlan anchor_plan(int B, int N, int H, int n_keys) {
+  AnchorPlan p;
+  const int Nk = n_keys > 0 ? n_keys : N;
+  p.n_qpairs = (N + 2 * BQ - 1) / (2 * BQ);
+  p.nkv_total = (Nk + BKV - 1) / BKV;
+  const int64_t units = static_cast<int64_t>(p.n_qpairs) * H * B;
+  const int sms = std::max(1, device_sm_count());  // one anchor CTA per SM
+  const int tail = static_cast<int>(units % sms);
+  p.n_full = static_cast<int>(units);
+  // The last wave's `tail` units, split s ways along the keys, take about
+  // ceil(tail * s / sms) / s of a whole unit's time. Take the best s <= 4 (and
+  // <= the key blocks) when it saves at least a fifth of that wave.
+  int best_s = 1;
+  double best_t = 1.0;
+  for (int sp = 2; sp <= std::min(4, p.nkv_total); ++sp) {
+    const double t = static_cast<double>((tail * sp + sms - 1) / sms) / sp;
+    if (t < best_t - 1e-9) {
+      best_t = t;
+      best_s = sp;
+    }
+  }
+  if (tail > 0 && best_s > 1 && best_t <= 0.8) {
+    p.split = best_s;
+    p.n_split_units = tail;
+    p.n_full = static_cast<int>(units - tail);
+  }
+  p.partial_bytes = static_cast<size_t>(p.n_split_units) * p.split * 2 * PART_FLOATS * sizeof(float);
+  return p;
+}
+
+cudaError_t anchor_bf16(const sva_attn_args& a, int* status, void* scratch, cudaStream_t s) {
   const int D = a.H * a.d;
   CUtensorMap mq, mk, mv;
   const int Nk = a.n_keys > 0 ? a.n_keys : a.N;
   if (!act_map(&mq, a.q, a.ldq, a.B, a.N, D) || !act_map(&mk, a.k, a.ldk, a.B, Nk, D) ||
       !act_map(&mv, a.v, a.ldv, a.B, Nk, D))
     return cudaErrorInvalidValue;
+  const AnchorPlan p = anchor_plan(a.B, a.N, a.H, a.n_keys);
+  if (p.partial_bytes > 0 && scratch == nullptr) return cudaErrorInvalidValue;
+  AnchorWork wk;
+  wk.n_qpairs = p.n_qpairs;
+  wk.H = a.H;
+  wk.n_full = p.n_full;
+  wk.n_split_units = p.n_split_units;
+  wk.split = p.split > 0 ? p.split : 1;
+  wk.nkv_total = p.nkv_total;
+  wk.partial = static_cast<float*>(scratch);
   const float scale = a.scale != 0.f ? a.scale : 1.0f / sqrtf(static_cast<float>(a.d));
   const float scale_log2 = scale * 1.4426950408889634f;
   cudaError_t e = cudaFuncSetAttribute(anchor_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(kAnchorSmem));
   if (e != cudaSuccess) return e;
-  dim3 grid((a.N + 2 * BQ - 1) / (2 * BQ), a.H, a.B);
-  anchor_tc_kernel<<<grid, NUM_THREADS, kAnchorSmem, s>>>(
-      mq, mk, mv, a.N, Nk, scale_log2, static_cast<const __nv_bfloat16*>(a.gate), a.ldg,
-      static_cast<const __nv_bfloat16*>(a.residual), a.ldr, static_cast<__nv_bfloat16*>(a.out),
-      a.ldo, status);
+  const unsigned grid = static_cast<unsigned>(p.n_full + p.n_split_units * p.split);
+  const auto* gate = static_cast<const __nv_bfloat16*>(a.gate);
+  const auto* res = static_cast<const __nv_bfloat16*>(a.residual);
+  auto* out = static_cast<__nv_bfloat16*>(a.out);
+  anchor_tc_kernel<<<grid, NUM_THREADS, kAnchorSmem, s>>>(mq, mk, mv, a.N, Nk, scale_log2, wk, gate,
+                                                          a.ldg, res, a.ldr, out, a.ldo, status);
+  if ((e = cudaGetLastError()) != cudaSuccess || p.n_split_units == 0) return e;
+  const int64_t threads = static_cast<int64_t>(p.n_split_units) * 2 * BQ * 32;
+  anchor_merge_kernel<<<static_cast<unsigned>((threads + 255) / 256), 256, 0, s>>>(
+      wk, a.N, gate, a.ldg, res, a.ldr, out, a.ldo);
   return cudaGetLastError();
 }
 

@@ -92,7 +92,14 @@ cudaError_t linear_f32(const sva_attn_args& a, int* status, void* scratch, cudaS
                        Prof* prof, float* state_out = nullptr, const float* state_in = nullptr);
 
 // ---------------------------------------------------------------- softmax anchor
-cudaError_t anchor_bf16(const sva_attn_args& a, int* status, cudaStream_t s);
+// Anchor launch plan: query-tile pairs, key blocks, and the split of the last
+// wave's units along the keys (partial_bytes of scratch for their parts).
+struct AnchorPlan {
+  int n_qpairs = 0, nkv_total = 0, n_full = 0, n_split_units = 0, split = 0;
+  size_t partial_bytes = 0;
+};
+AnchorPlan anchor_plan(int B, int N, int H, int n_keys);
+cudaError_t anchor_bf16(const sva_attn_args& a, int* status, void* scratch, cudaStream_t s);
 cudaError_t anchor_f32(const sva_attn_args& a, int* status, cudaStream_t s);
 
 // ---------------------------------------------------------------- router

@@ -211,20 +211,29 @@ extern "C" sva_status_t sva_linear_attn_readout_fwd(const sva_attn_args* args, c
   return e == cudaSuccess ? SVA_OK : cuda_fail(e);
 }
 
-extern "C" size_t sva_softmax_anchor_workspace_bytes(int, int, int, int, sva_dtype_t) {
-  return SVA_STATUS_BYTES;
+extern "C" size_t sva_softmax_anchor_workspace_bytes(int B, int N, int H, int d,
+                                                     sva_dtype_t dtype) {
+  if (B < 1 || N < 1 || H < 1 || d < 1) return 0;
+  if (dtype != SVA_BF16) return SVA_STATUS_BYTES;
+  // the split parts of the last wave (bounded over every key count)
+  return SVA_STATUS_BYTES + anchor_plan(B, N, H, 1 << 30).partial_bytes;
 }
 
 extern "C" sva_status_t sva_softmax_anchor_fwd(const sva_attn_args* args, void* ws, size_t ws_bytes,
                                                sva_stream_t stream) {
   sva_status_t st = check_attn(args, false);
   if (st != SVA_OK) return st;
-  if (ws == nullptr || !aligned16(ws) || ws_bytes < SVA_STATUS_BYTES) return SVA_ERR_WORKSPACE;
+  const size_t need =
+      SVA_STATUS_BYTES +
+      (args->dtype == SVA_BF16 ? anchor_plan(args->B, args->N, args->H, args->n_keys).partial_bytes
+                               : 0);
+  if (ws == nullptr || !aligned16(ws) || ws_bytes < need) return SVA_ERR_WORKSPACE;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   if ((st = clear_status(ws, s)) != SVA_OK) return st;
   int* status = static_cast<int*>(ws);
-  cudaError_t e = args->dtype == SVA_BF16 ? anchor_bf16(*args, status, s)
-                                          : anchor_f32(*args, status, s);
+  cudaError_t e = args->dtype == SVA_BF16
+                      ? anchor_bf16(*args, status, static_cast<char*>(ws) + SVA_STATUS_BYTES, s)
+                      : anchor_f32(*args, status, s);
   return e == cudaSuccess ? SVA_OK : cuda_fail(e);
 }
 
@@ -387,7 +396,9 @@ StackLayout stack_layout(const sva_stack_desc& d) {
   s.u = take(rows * D * es);
   s.qkvg = take(rows * static_cast<size_t>(qkvg_ld(d)) * es);
   s.y = take(rows * D * es);
-  s.lin = take(linear_plan(d.B, d.N, d.H, d.d, d.dtype).total);
+  // attention scratch: the linear layers' partial states, or the anchors' split parts
+  s.lin = take(std::max(linear_plan(d.B, d.N, d.H, d.d, d.dtype).total,
+                        d.dtype == SVA_BF16 ? anchor_plan(d.B, d.N, d.H, 0).partial_bytes : 0));
   s.n_summ = summaries_needed(d);
   s.wrt = take(s.n_summ > 0 ? D * D * es : 0);
   s.summ = take(static_cast<size_t>(s.n_summ) * rows * D * es);
@@ -534,7 +545,7 @@ sva_status_t stack_pass(const sva_stack_desc* desc, const void* x, void* y, void
     }
     if (anchor) {
       ProfScope ps(prof, s, SVA_KERNEL_ANCHOR);
-      SVA_TRY(bf16 ? anchor_bf16(a, status, s) : anchor_f32(a, status, s));
+      SVA_TRY(bf16 ? anchor_bf16(a, status, lin_scratch, s) : anchor_f32(a, status, s));
     } else {
       SVA_TRY(bf16 ? linear_bf16(a, status, lin_scratch, s, prof)
                    : linear_f32(a, status, lin_scratch, s, prof));

@@ -354,7 +354,7 @@ def timed_steps(torch, sva, stack, x, y, ws, steps, profile=True):
         del probe
     start = torch.cuda.Event(enable_timing=True)
     end = torch.cuda.Event(enable_timing=True)
-    counts, kinds = [], []
+    counts, kinds, kernels = [], [], 0
     start.record(stream)
     for k in range(steps):
         if profile:
@@ -363,17 +363,16 @@ def timed_steps(torch, sva, stack, x, y, ws, steps, profile=True):
         if profile:
             counts.append(stack.prof_count.value)
             kinds.append(list(stack.prof_kind))
+            kernels += stack.launch_count.value  # a profiled span may hold 2 kernels
     end.record(stream)
     torch.cuda.synchronize()
     stack.clear_profile()
     recs = []
-    launches = 0
     for k in range(len(counts)):
         n = min(counts[k], len(ev_sets[k]) // 2)
-        launches += counts[k]
         for i in range(n):
             recs.append((KINDS[kinds[k][i]], ev_sets[k][2 * i].elapsed_time(ev_sets[k][2 * i + 1])))
-    return start.elapsed_time(end), recs, launches
+    return start.elapsed_time(end), recs, kernels
 
 
 def summarize(recs, steps, wl, peaks):

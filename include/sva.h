@@ -258,6 +258,8 @@ typedef struct {
   int* prof_kind;              /* optional host array [prof_capacity]            */
   int* prof_count;             /* optional host int                              */
   const void* const* w_wg;     /* optional, L pointers, each [H, D] in dtype     */
+  int* launch_count;           /* optional host int: kernels the call launched
+                                  (counted while profiling, prof_events set)    */
 } sva_stack_desc;
 
 size_t sva_hybrid_stack_workspace_bytes(const sva_stack_desc* desc);

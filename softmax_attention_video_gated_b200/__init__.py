@@ -65,6 +65,7 @@ class StackDesc(ctypes.Structure):
         ("prof_events", _c_void_p_p), ("prof_capacity", ctypes.c_int),
         ("prof_kind", ctypes.POINTER(ctypes.c_int)), ("prof_count", ctypes.POINTER(ctypes.c_int)),
         ("w_wg", _c_void_p_p),
+        ("launch_count", ctypes.POINTER(ctypes.c_int)),
     ]
 
 
@@ -394,6 +395,7 @@ class Stack:
         self.desc = d
         self.tensors = (w_qkvg, w_o, w_r, trace_o, trace_y, trace_alpha, w_wg)
         self.prof_count = ctypes.c_int(0)
+        self.launch_count = ctypes.c_int(0)
 
     def set_profile(self, events: Sequence, kinds_capacity: int):
         """events: 2*capacity torch.cuda.Event(enable_timing=True), already recorded once."""
@@ -405,12 +407,14 @@ class Stack:
         self.desc.prof_capacity = cap
         self.desc.prof_kind = ctypes.cast(self.prof_kind, ctypes.POINTER(ctypes.c_int))
         self.desc.prof_count = ctypes.pointer(self.prof_count)
+        self.desc.launch_count = ctypes.pointer(self.launch_count)
 
     def clear_profile(self):
         self.desc.prof_events = None
         self.desc.prof_capacity = 0
         self.desc.prof_kind = None
         self.desc.prof_count = None
+        self.desc.launch_count = None
 
     def workspace_bytes(self) -> int:
         n = int(_lib().sva_hybrid_stack_workspace_bytes(ctypes.byref(self.desc)))

@@ -579,7 +579,8 @@ AnchorPlan anchor_plan(int B, int N, int H, int n_keys) {
   return p;
 }
 
-cudaError_t anchor_bf16(const sva_attn_args& a, int* status, void* scratch, cudaStream_t s) {
+cudaError_t anchor_bf16(const sva_attn_args& a, int* status, void* scratch, cudaStream_t s,
+                        Prof* prof) {
   const int D = a.H * a.d;
   CUtensorMap mq, mk, mv;
   const int Nk = a.n_keys > 0 ? a.n_keys : a.N;
@@ -611,6 +612,7 @@ cudaError_t anchor_bf16(const sva_attn_args& a, int* status, void* scratch, cuda
   const int64_t threads = static_cast<int64_t>(p.n_split_units) * 2 * BQ * 32;
   anchor_merge_kernel<<<static_cast<unsigned>((threads + 255) / 256), 256, 0, s>>>(
       wk, a.N, gate, a.ldg, res, a.ldr, out, a.ldo);
+  if (prof != nullptr) prof->extra_launch();
   return cudaGetLastError();
 }
 

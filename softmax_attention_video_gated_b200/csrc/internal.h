@@ -15,6 +15,7 @@ struct Prof {
   int capacity = 0;
   int* kinds = nullptr;           // host, capacity
   int count = 0;
+  int launches = 0;  // kernels launched (a scope may launch more than one)
   int cur_kind = SVA_KERNEL_OTHER;
   void before(cudaStream_t s, int kind) {
     cur_kind = kind;
@@ -26,7 +27,9 @@ struct Prof {
       if (kinds != nullptr) kinds[count] = cur_kind;
     }
     ++count;
+    ++launches;
   }
+  void extra_launch() { ++launches; }  // a second kernel inside one scope
 };
 
 struct ProfScope {
@@ -99,7 +102,8 @@ struct AnchorPlan {
   size_t partial_bytes = 0;
 };
 AnchorPlan anchor_plan(int B, int N, int H, int n_keys);
-cudaError_t anchor_bf16(const sva_attn_args& a, int* status, void* scratch, cudaStream_t s);
+cudaError_t anchor_bf16(const sva_attn_args& a, int* status, void* scratch, cudaStream_t s,
+                        Prof* prof = nullptr);
 cudaError_t anchor_f32(const sva_attn_args& a, int* status, cudaStream_t s);
 
 // ---------------------------------------------------------------- router

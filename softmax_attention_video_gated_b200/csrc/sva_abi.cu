@@ -545,7 +545,7 @@ sva_status_t stack_pass(const sva_stack_desc* desc, const void* x, void* y, void
     }
     if (anchor) {
       ProfScope ps(prof, s, SVA_KERNEL_ANCHOR);
-      SVA_TRY(bf16 ? anchor_bf16(a, status, lin_scratch, s) : anchor_f32(a, status, s));
+      SVA_TRY(bf16 ? anchor_bf16(a, status, lin_scratch, s, prof) : anchor_f32(a, status, s));
     } else {
       SVA_TRY(bf16 ? linear_bf16(a, status, lin_scratch, s, prof)
                    : linear_f32(a, status, lin_scratch, s, prof));
@@ -590,6 +590,7 @@ sva_status_t stack_pass(const sva_stack_desc* desc, const void* x, void* y, void
   }
 #undef SVA_TRY
   if (d.prof_count != nullptr) *d.prof_count = prof != nullptr ? prof->count : 0;
+  if (d.launch_count != nullptr) *d.launch_count = prof != nullptr ? prof->launches : 0;
   return SVA_OK;
 }
 

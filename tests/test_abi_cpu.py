@@ -89,6 +89,21 @@ def test_phase_and_key_count_host_validation():
                                       None) == sva.SVA_ERR_INVALID_ARGUMENT
 
 
+def test_sizes_past_the_index_range_are_refused_on_host():
+    # token counts and GEMM extents are indexed in 32 bits inside the kernels:
+    # B*N, B*n_keys or an extent above 2^31 is refused before anything launches
+    lib = sva._lib()
+    a = _args(B=3, N=1 << 30)
+    assert lib.sva_linear_attn_fwd(ctypes.byref(a), 0x20000, 1 << 62, None) == sva.SVA_ERR_UNSUPPORTED
+    assert lib.sva_softmax_anchor_fwd(ctypes.byref(a), 0x20000, 1 << 62,
+                                      None) == sva.SVA_ERR_UNSUPPORTED
+    a = _args(B=3, N=1000, n_keys=1 << 30)
+    assert lib.sva_softmax_anchor_fwd(ctypes.byref(a), 0x20000, 1 << 62,
+                                      None) == sva.SVA_ERR_UNSUPPORTED
+    assert lib.sva_projection_fwd(0x10000, 64, 0x20000, (1 << 31) + 1, 64, 64, 0x30000, 64, 0,
+                                  sva.SVA_BF16, 0x40000, 256, None) == sva.SVA_ERR_UNSUPPORTED
+
+
 def test_workspace_checks_happen_before_launch():
     a = _args()
     assert sva._lib().sva_linear_attn_fwd(ctypes.byref(a), None, 0, None) == sva.SVA_ERR_WORKSPACE

@@ -28,16 +28,19 @@
 // pairs (one f32x2 FFMA or FADD per two keys). Exponentials run on the MUFU
 // unit; kPolyEvery can send every k-th one to the FMA pipe instead (Cody-Waite
 // reduction and a minimax cubic, see fit_exp2_poly.py).
-// What bounds it (720p layer on B200, clock64 traces of one CTA): the softmax
-// warps wait for S about half of each 128-key step; the MMA thread issues
-// without pause, each 128x128x16 MMA taking ~88 cycles with both operands in
-// shared memory and ~59 with P in TMEM, and the tensor pipe drains while that
-// thread waits on barriers between MMA groups. Measured: 4.02 ms with packed
-// pairs, 4.35 ms without; sending one exponential pair in eight, four or three
-// to the FMA pipe: 4.10, 4.33, 4.52 ms; MMAs alone (no softmax dependency):
-// 3.10 ms. The wait for K_{j+1} sat after the first tile's P V issue so it
-// overlaps that MMA; then 3.94 ms once the waits for V_j and K_{j+1} moved
-// from the MMA thread to a softmax warp of each tile.
+// What bounds it (720p layer on B200, clock64 traces of one CTA, ncu): each
+// tile's chain -- softmax of block j (about 2,100 cycles, 1,260 of them on the
+// exponentials), then P_j V_j and S_{j+1} on the tensor core (about 1,250),
+// then the wake-ups -- sets the step at about 3,700 cycles for two tiles, and
+// the tensor and MUFU pipes are each active about half of the time. Alone, a
+// 128x128x16 MMA takes its nominal 64 cycles in every form used here (also
+// back to back on aliased columns, and with other warps reading TMEM); inside
+// the kernel the MMA thread shares its SM sub-partition with two busy softmax
+// warps, so its own instruction count sets how fast MMAs are issued: its
+// shared-memory descriptors are therefore built once and offset by constants
+// (8,190 keys: 0.87 -> 0.79 ms; 720p: 3.94 -> 3.90 ms). Earlier steps:
+// packed pairs 4.35 -> 4.02 ms; the waits for V_j and K_{j+1} moved from the
+// MMA thread to a softmax warp of each tile, 3.94 ms.
 #include <algorithm>
 #include <math.h>
 
@@ -124,7 +127,7 @@ __device__ __forceinline__ float ex2_row(float x, int idx) {
 // (merge included, 14 us) from 3.96-4.01 to 3.95-3.99 ms. It pays most when
 // a call has fewer units than SMs.
 struct AnchorWork {
-  int n_qpairs, H, n_full, n_split_units, split, nkv_total;
+  int n_qunits, H, n_full, n_split_units, split, nkv_total;
   float* partial;  // [n_split_units][split][2 tiles][BQ x HD O | BQ x (m, l)]
 };
 constexpr int PART_FLOATS = BQ * HD + 2 * BQ;
@@ -150,8 +153,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     kb0 = part * wk.nkv_total / wk.split;
     nkv = (part + 1) * wk.nkv_total / wk.split - kb0;
   }
-  const int q0 = (unit % wk.n_qpairs) * 2 * BQ;
-  const int h = (unit / wk.n_qpairs) % wk.H, b = unit / (wk.n_qpairs * wk.H);
+  const int q0 = (unit % wk.n_qunits) * 2 * BQ;
+  const int h = (unit / wk.n_qunits) % wk.H, b = unit / (wk.n_qunits * wk.H);
   const int warp = warp_id(), lane = lane_id();
   const int wg = warp >> 2;
   const bool has1 = q0 + BQ < N;  // the second tile holds at least one query
@@ -246,27 +249,31 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       constexpr uint32_t idesc_o = idesc_bf16_f32(BQ, HD, false, true);    // P (TMEM), V: MN-major
       const int ntiles = has1 ? 2 : 1;
       bool ok = mbar_wait(&tl->q_full, 0, abort_flag, status, WHERE_ANCHOR);
-      auto issue_s = [&](int t, int j) {
-        const uint32_t qaddr = smem_u32(smem + Q_OFF + t * 2 * BOX);
-        const uint32_t kaddr = smem_u32(smem + K_OFF + (j % K_STAGES) * 2 * BOX);
+      // The MMA thread shares its SM sub-partition with two softmax warps, so
+      // its own instruction count is on the critical path: descriptors are
+      // built once and each MMA adds a compile-time offset to a stage's base
+      // (start addresses stay below 256 KB, so the 14-bit field never carries).
+      const uint64_t qd0 = smem_desc(smem_u32(smem + Q_OFF), 16, 1024);
+      const uint64_t kd0 = smem_desc(smem_u32(smem + K_OFF), 16, 1024);
+      const uint64_t vd0 = smem_desc(smem_u32(smem + V_OFF), BOX, 1024);
+      auto issue_s = [&](int t, int kst) {
+        const uint64_t qb = qd0 + static_cast<uint64_t>(t * (2 * BOX >> 4));
+        const uint64_t kb = kd0 + static_cast<uint64_t>(kst * (2 * BOX >> 4));
         const uint32_t d_tmem = tmem + t * 256;
 #pragma unroll
         for (int kk = 0; kk < HD / 16; ++kk) {
-          const int bx = kk >> 2, w = kk & 3;
-          const uint64_t ad = smem_desc(qaddr + bx * BOX + w * 32, 16, 1024);
-          const uint64_t bd = smem_desc(kaddr + bx * BOX + w * 32, 16, 1024);
-          umma_ss(d_tmem, ad, bd, idesc_s, kk != 0 ? 1u : 0u);
+          const uint32_t off = static_cast<uint32_t>(((kk >> 2) * BOX + (kk & 3) * 32) >> 4);
+          umma_ss(d_tmem, qb + off, kb + off, idesc_s, kk != 0 ? 1u : 0u);
         }
         umma_commit(&tl->s_full[t]);
       };
-      auto issue_pv = [&](int t, int j) {
-        const uint32_t vaddr = smem_u32(smem + V_OFF + (j % V_STAGES) * 2 * BOX);
+      auto issue_pv = [&](int t, int vst, bool first) {
+        const uint64_t vb = vd0 + static_cast<uint64_t>(vst * (2 * BOX >> 4));
         const uint32_t p_tmem = tmem + t * 256;
 #pragma unroll
-        for (int kk = 0; kk < BKV / 16; ++kk) {
-          const uint64_t bd = smem_desc(vaddr + kk * 2048, BOX, 1024);
-          umma_ts(tmem + t * 256 + 128, p_tmem + kk * 8, bd, idesc_o, (j | kk) != 0 ? 1u : 0u);
-        }
+        for (int kk = 0; kk < BKV / 16; ++kk)
+          umma_ts(p_tmem + 128, p_tmem + kk * 8, vb + static_cast<uint32_t>(kk * 2048 >> 4), idesc_o,
+                  (kk != 0 || !first) ? 1u : 0u);
       };
       if (ok && nkv > 0) {
         ok = mbar_wait(&tl->k_full[0], 0, abort_flag, status, WHERE_ANCHOR);
@@ -276,9 +283,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           umma_commit(&tl->k_empty[0]);
         }
       }
+      int vst = 0, kn = 1 % K_STAGES;  // stages of V_j and K_{j+1}
       for (int j = 0; j < nkv && ok; ++j) {
         const bool more = j + 1 < nkv;
-        const int kn = (j + 1) % K_STAGES;
         // V_j and K_{j+1} need no wait here: a softmax warp of each tile saw
         // them land before it reported P_j (its p_full arrival orders them)
         for (int t = 0; t < ntiles; ++t) {
@@ -287,13 +294,15 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             break;
           }
           tc_fence_after();
-          issue_pv(t, j);
-          if (t == ntiles - 1) umma_commit(&tl->v_empty[j % V_STAGES]);
+          issue_pv(t, vst, j == 0);
+          if (t == ntiles - 1) umma_commit(&tl->v_empty[vst]);
           if (more) {
-            issue_s(t, j + 1);
+            issue_s(t, kn);
             if (t == ntiles - 1) umma_commit(&tl->k_empty[kn]);
           }
         }
+        vst = vst + 1 == V_STAGES ? 0 : vst + 1;
+        kn = kn + 1 == K_STAGES ? 0 : kn + 1;
       }
       if (ok) umma_commit(&tl->o_done);
       umma_commit(&tl->drain);
@@ -498,8 +507,8 @@ __global__ void __launch_bounds__(256) anchor_merge_kernel(AnchorWork wk, int N,
   const int su = static_cast<int>(wid / (2 * BQ));
   const int t = static_cast<int>((wid / BQ) & 1), r = static_cast<int>(wid % BQ);
   const int unit = wk.n_full + su;
-  const int q0 = (unit % wk.n_qpairs) * 2 * BQ;
-  const int h = (unit / wk.n_qpairs) % wk.H, b = unit / (wk.n_qpairs * wk.H);
+  const int q0 = (unit % wk.n_qunits) * 2 * BQ;
+  const int h = (unit / wk.n_qunits) % wk.H, b = unit / (wk.n_qunits * wk.H);
   const int row_t = q0 + t * BQ + r;
   if (row_t >= N) return;
   float mx = -INFINITY;
@@ -552,9 +561,9 @@ bool act_map(CUtensorMap* m, const void* base, int64_t ld, int B, int N, int D) 
 AnchorPlan anchor_plan(int B, int N, int H, int n_keys) {
   AnchorPlan p;
   const int Nk = n_keys > 0 ? n_keys : N;
-  p.n_qpairs = (N + 2 * BQ - 1) / (2 * BQ);
+  p.n_qunits = (N + 2 * BQ - 1) / (2 * BQ);
   p.nkv_total = (Nk + BKV - 1) / BKV;
-  const int64_t units = static_cast<int64_t>(p.n_qpairs) * H * B;
+  const int64_t units = static_cast<int64_t>(p.n_qunits) * H * B;
   const int sms = std::max(1, device_sm_count());  // one anchor CTA per SM
   const int tail = static_cast<int>(units % sms);
   p.n_full = static_cast<int>(units);
@@ -590,7 +599,7 @@ cudaError_t anchor_bf16(const sva_attn_args& a, int* status, void* scratch, cuda
   const AnchorPlan p = anchor_plan(a.B, a.N, a.H, a.n_keys);
   if (p.partial_bytes > 0 && scratch == nullptr) return cudaErrorInvalidValue;
   AnchorWork wk;
-  wk.n_qpairs = p.n_qpairs;
+  wk.n_qunits = p.n_qunits;
   wk.H = a.H;
   wk.n_full = p.n_full;
   wk.n_split_units = p.n_split_units;

@@ -95,10 +95,11 @@ cudaError_t linear_f32(const sva_attn_args& a, int* status, void* scratch, cudaS
                        Prof* prof, float* state_out = nullptr, const float* state_in = nullptr);
 
 // ---------------------------------------------------------------- softmax anchor
-// Anchor launch plan: query-tile pairs, key blocks, and the split of the last
-// wave's units along the keys (partial_bytes of scratch for their parts).
+// Anchor launch plan: units of 512 queries (one CTA pair each), key blocks,
+// and the split of the last wave's units along the keys (partial_bytes of
+// scratch for their parts).
 struct AnchorPlan {
-  int n_qpairs = 0, nkv_total = 0, n_full = 0, n_split_units = 0, split = 0;
+  int n_qunits = 0, nkv_total = 0, n_full = 0, n_split_units = 0, split = 0;
   size_t partial_bytes = 0;
 };
 AnchorPlan anchor_plan(int B, int N, int H, int n_keys);

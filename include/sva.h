@@ -32,7 +32,7 @@
  *    SVA_ERR_DEVICE_TIMEOUT there and returns (no trap). Read it with
  *    sva_check_device_status.
  *  - Errors: SVA_ERR_INVALID_ARGUMENT (null pointer, bad size, stride or
- *    alignment), SVA_ERR_UNSUPPORTED (a valid shape this build has no kernel
+ *    alignment), SVA_ERR_UNSUPPORTED (a valid shape the library has no kernel
  *    for, e.g. bf16 with d != 128), SVA_ERR_WORKSPACE (ws too small),
  *    SVA_ERR_CUDA (a launch or runtime call failed; see sva_last_cuda_error).
  */

@@ -7,9 +7,9 @@
 // CTA r loads rows [128r, 128r+128) of the A tile and rows [128r, 128r+128) of
 // the B tile (its half of N), so a k-block costs each CTA 32 KB of shared
 // memory instead of the 48 KB a single-CTA 128 x 256 tile needs. Per CTA:
-//   warp 0      TMA producer: 128x64 A and 128x64 B boxes (128-byte swizzle)
-//               into a 6-stage ring; completion is counted on the rank-0 CTA's
-//               barrier, which expects both CTAs' bytes;
+//   warp 0      TMA producer: 128-row A and B boxes of 64 columns (128-byte
+//               swizzle) into a ring of k-blocks; completion is counted on the
+//               rank-0 CTA's barrier, which expects both CTAs' bytes;
 //   warp 1      allocates 512 TMEM columns (pair allocation); on rank 0 one
 //               lane issues M=256 N=256 K=16 MMAs into one of two 256-column
 //               accumulators and multicasts its commits to both CTAs;
@@ -19,6 +19,13 @@
 //               the feature map phi of the linear layers) or the residual
 //               update h += C (fp32) with an optional bf16 copy of h. Each warp
 //               releases the accumulator on rank 0's barrier.
+// A k-block is 128 deep (two boxes per operand, 3 stages) for the bf16 store
+// epilogue and 64 deep (5 stages) for the residual one, whose h buffers leave
+// no room for a third 64 KB stage. Every k-block costs the MMA thread one
+// barrier wait and one commit, and those stall its queue of MMAs, so deeper
+// k-blocks pay off where three stages fit: the 720p QKVG projection takes
+// 0.91 ms instead of 0.96 ms; the residual GEMM with 2 such stages was 20%
+// slower than with five of 64.
 // Tiles run in groups of whole M-tile columns so one wave touches few A rows
 // and few B rows and both stay in L2. A ragged last N tile issues MMAs only as
 // wide as its columns (rounded up to 32), and the output columns from n_split
@@ -32,11 +39,9 @@
 namespace sva {
 namespace {
 
-constexpr int BM = 256, BN = 256, BK = 64, MAX_STAGES = 6;
+constexpr int BM = 256, BN = 256, MAX_STAGES = 5;
 constexpr int HALF = 128;                          // rows of A (and of B) per CTA
-constexpr int A_STAGE = HALF * BK * 2;             // 16 KB
-constexpr int B_STAGE = HALF * BK * 2;             // 16 KB
-constexpr int STAGE_BYTES = A_STAGE + B_STAGE;     // 32 KB per CTA
+constexpr int KBOX = HALF * 64 * 2;                // one 128 x 64 bf16 box: 16 KB
 constexpr int TMEM_COLS = 2 * BN;                  // two fp32 accumulators
 constexpr int NUM_THREADS = 192;
 // EPI_STORE epilogue: a 32 x 32 fp32 transpose buffer per warp
@@ -49,7 +54,10 @@ constexpr int RES_WARP_BYTES = 2 * RES_H_BYTES + 2 * RES_C_BYTES;  // 12 KB
 
 template <int EPI>
 struct Layout {
-  static constexpr int STAGES = EPI == EPI_STORE ? 6 : 5;
+  static constexpr int BK = EPI == EPI_STORE ? 128 : 64;      // k-block depth
+  static constexpr int STAGES = EPI == EPI_STORE ? 3 : 5;
+  static constexpr int A_STAGE = HALF * BK * 2;                // 32 or 16 KB
+  static constexpr int STAGE_BYTES = 2 * A_STAGE;              // A and B, per CTA
   static constexpr int EPI_OFF = STAGES * STAGE_BYTES;
   static constexpr int TAIL_OFF = EPI_OFF + 4 * (EPI == EPI_STORE ? STG_WARP_BYTES : RES_WARP_BYTES);
 };
@@ -100,7 +108,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                         const __grid_constant__ CUtensorMap map_b2,
                         const __grid_constant__ CUtensorMap map_h,
                         const __grid_constant__ CUtensorMap map_c, GemmArgs g, int group) {
-  constexpr int STAGES = Layout<EPI>::STAGES;
+  constexpr int STAGES = Layout<EPI>::STAGES, BK = Layout<EPI>::BK;
+  constexpr int A_STAGE = Layout<EPI>::A_STAGE, B_STAGE = A_STAGE;
+  constexpr int STAGE_BYTES = Layout<EPI>::STAGE_BYTES;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
@@ -173,8 +183,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           }
           const uint32_t full0 = cluster_map(&tl->full[stage], 0);
           if (rank == 0) mbar_arrive_expect_tx(&tl->full[stage], 2 * STAGE_BYTES);
-          tma_load_2d_pair(&map_a, full0, sA + stage * A_STAGE, kb * BK, m_blk * BM + rank * HALF);
-          tma_load_2d_pair(mb, full0, sB + stage * B_STAGE, kb * BK, b_row);
+#pragma unroll
+          for (int bx = 0; bx < BK / 64; ++bx) {
+            tma_load_2d_pair(&map_a, full0, sA + stage * A_STAGE + bx * KBOX, kb * BK + 64 * bx,
+                             m_blk * BM + rank * HALF);
+            tma_load_2d_pair(mb, full0, sB + stage * B_STAGE + bx * KBOX, kb * BK + 64 * bx, b_row);
+          }
           ++issued;
           if (++stage == STAGES) {
             stage = 0;
@@ -218,8 +232,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           const uint32_t b_addr = smem_u32(sB + stage * B_STAGE);
 #pragma unroll
           for (int kk = 0; kk < BK / 16; ++kk) {
-            const uint64_t ad = smem_desc(a_addr + kk * 32, 16, 1024);
-            const uint64_t bd = smem_desc(b_addr + kk * 32, 16, 1024);
+            const uint32_t off = static_cast<uint32_t>((kk >> 2) * KBOX + (kk & 3) * 32);
+            const uint64_t ad = smem_desc(a_addr + off, 16, 1024);
+            const uint64_t bd = smem_desc(b_addr + off, 16, 1024);
             umma_ss_pair(d_tmem, ad, bd, idesc, (kb | kk) != 0 ? 1u : 0u);
           }
           umma_commit_pair(&tl->empty[stage], 0x3);
@@ -437,7 +452,7 @@ cudaError_t gemm_bf16(const GemmArgs& g, cudaStream_t s) {
   {
     const uint64_t dims[2] = {static_cast<uint64_t>(g.K), static_cast<uint64_t>(g.M)};
     const uint64_t strides[1] = {static_cast<uint64_t>(g.lda) * 2};
-    const uint32_t box[2] = {BK, HALF};
+    const uint32_t box[2] = {64, HALF};
     if (!encode_tmap(&ma, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, g.a, dims, strides, box,
                      CU_TENSOR_MAP_SWIZZLE_128B))
       return cudaErrorInvalidValue;
@@ -448,7 +463,7 @@ cudaError_t gemm_bf16(const GemmArgs& g, cudaStream_t s) {
   {
     const uint64_t dims[2] = {static_cast<uint64_t>(g.K), static_cast<uint64_t>(n_first)};
     const uint64_t strides[1] = {static_cast<uint64_t>(g.ldb) * 2};
-    const uint32_t box[2] = {BK, HALF};
+    const uint32_t box[2] = {64, HALF};
     if (!encode_tmap(&mb, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, g.b, dims, strides, box,
                      CU_TENSOR_MAP_SWIZZLE_128B))
       return cudaErrorInvalidValue;
@@ -457,7 +472,7 @@ cudaError_t gemm_bf16(const GemmArgs& g, cudaStream_t s) {
   if (g.b2 != nullptr) {
     const uint64_t dims[2] = {static_cast<uint64_t>(g.K), static_cast<uint64_t>(g.N - g.n_split)};
     const uint64_t strides[1] = {static_cast<uint64_t>(g.ldb) * 2};
-    const uint32_t box[2] = {BK, HALF};
+    const uint32_t box[2] = {64, HALF};
     if (!encode_tmap(&mb2, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, g.b2, dims, strides, box,
                      CU_TENSOR_MAP_SWIZZLE_128B))
       return cudaErrorInvalidValue;

@@ -19,13 +19,13 @@
 //               the feature map phi of the linear layers) or the residual
 //               update h += C (fp32) with an optional bf16 copy of h. Each warp
 //               releases the accumulator on rank 0's barrier.
-// A k-block is 128 deep (two boxes per operand, 3 stages) for the bf16 store
-// epilogue and 64 deep (5 stages) for the residual one, whose h buffers leave
-// no room for a third 64 KB stage. Every k-block costs the MMA thread one
-// barrier wait and one commit, and those stall its queue of MMAs, so deeper
-// k-blocks pay off where three stages fit: the 720p QKVG projection takes
-// 0.91 ms instead of 0.96 ms; the residual GEMM with 2 such stages was 20%
-// slower than with five of 64.
+// A k-block is 128 deep (two boxes per operand) in a 3-stage ring. Every
+// k-block costs the MMA thread one barrier wait and one commit, and those
+// stall its queue of MMAs, so 8 MMAs per k-block run faster than 4: the 720p
+// QKVG projection takes 0.91 ms instead of 0.96 ms with 64-deep k-blocks. The
+// residual epilogue moves h in 16-column chunks (6 KB of slots per warp) so
+// that three 64 KB stages fit beside it (0.297 against 0.302 ms at 720p with
+// 32-column chunks and five 32 KB stages).
 // Tiles run in groups of whole M-tile columns so one wave touches few A rows
 // and few B rows and both stay in L2. A ragged last N tile issues MMAs only as
 // wide as its columns (rounded up to 32), and the output columns from n_split
@@ -39,7 +39,7 @@
 namespace sva {
 namespace {
 
-constexpr int BM = 256, BN = 256, MAX_STAGES = 5;
+constexpr int BM = 256, BN = 256, MAX_STAGES = 3;
 constexpr int HALF = 128;                          // rows of A (and of B) per CTA
 constexpr int KBOX = HALF * 64 * 2;                // one 128 x 64 bf16 box: 16 KB
 constexpr int TMEM_COLS = 2 * BN;                  // two fp32 accumulators
@@ -47,18 +47,20 @@ constexpr int NUM_THREADS = 192;
 // EPI_STORE epilogue: a 32 x 32 fp32 transpose buffer per warp
 constexpr int STG_STRIDE = 36;                     // fp32 words per staged row (16-byte aligned)
 constexpr int STG_WARP_BYTES = 32 * STG_STRIDE * 4;
-// EPI_RESIDUAL epilogue: per warp two slots of a 32 x 32 fp32 tile of h
-// (128-byte swizzle) and two of its 32 x 32 bf16 copy (64-byte swizzle)
-constexpr int RES_H_BYTES = 32 * 32 * 4, RES_C_BYTES = 32 * 32 * 2;
-constexpr int RES_WARP_BYTES = 2 * RES_H_BYTES + 2 * RES_C_BYTES;  // 12 KB
+// EPI_RESIDUAL epilogue: per warp two slots of a 32-row x 16-column fp32 chunk
+// of h (64-byte swizzle) and two of its bf16 copy (32-byte swizzle)
+constexpr int RES_COLS = 16;                       // columns of h per chunk
+constexpr int RES_H_BYTES = 32 * RES_COLS * 4, RES_C_BYTES = 32 * RES_COLS * 2;
+constexpr int RES_WARP_BYTES = 2 * RES_H_BYTES + 2 * RES_C_BYTES;  // 6 KB
 
 template <int EPI>
 struct Layout {
-  static constexpr int BK = EPI == EPI_STORE ? 128 : 64;      // k-block depth
-  static constexpr int STAGES = EPI == EPI_STORE ? 3 : 5;
-  static constexpr int A_STAGE = HALF * BK * 2;                // 32 or 16 KB
+  static constexpr int BK = 128;                              // k-block depth
+  static constexpr int STAGES = 3;
+  static constexpr int A_STAGE = HALF * BK * 2;                // 32 KB
   static constexpr int STAGE_BYTES = 2 * A_STAGE;              // A and B, per CTA
   static constexpr int EPI_OFF = STAGES * STAGE_BYTES;
+  static_assert(STAGES <= MAX_STAGES, "barrier arrays hold every stage");
   static constexpr int TAIL_OFF = EPI_OFF + 4 * (EPI == EPI_STORE ? STG_WARP_BYTES : RES_WARP_BYTES);
 };
 
@@ -312,8 +314,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     }
   } else {
     // ------------------------------------------------ residual epilogue (warps 2..5, both CTAs)
-    // h += C for this warp's 32 rows, 32 columns at a time: TMA brings the h
-    // chunk into a 128-byte-swizzled slot (prefetched two chunks ahead), the
+    // h += C for this warp's 32 rows, 16 columns at a time: TMA brings the h
+    // chunk into a 64-byte-swizzled slot (prefetched two chunks ahead), the
     // thread owning a row adds its accumulator row in place (the swizzle keeps
     // the row-per-thread access free of bank conflicts), and TMA writes h and
     // its bf16 copy back.
@@ -334,13 +336,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       tile_coords(tile, m_tiles, n_tiles, group, m_blk, n_blk);
       const int64_t row0 = static_cast<int64_t>(m_blk) * BM + rank * HALF + q * 32;
       const int64_t colT = static_cast<int64_t>(n_blk) * BN;
-      const int64_t left = (g.N - colT + 31) / 32;
-      const int nch = row0 < g.M ? static_cast<int>(left < 8 ? left : 8) : 0;
+      const int64_t left = (g.N - colT + RES_COLS - 1) / RES_COLS;
+      const int nch = row0 < g.M ? static_cast<int>(left < BN / RES_COLS ? left : BN / RES_COLS) : 0;
       if (lane == 0) {
         tma_store_wait_read0();  // both slots free again
         for (int c = 0; c < min(2, nch); ++c) {
           mbar_arrive_expect_tx(&hbar[c], RES_H_BYTES);
-          tma_load_2d(&map_h, &hbar[c], wbuf + c * RES_H_BYTES, static_cast<int>(colT + 32 * c),
+          tma_load_2d(&map_h, &hbar[c], wbuf + c * RES_H_BYTES, static_cast<int>(colT + RES_COLS * c),
                       static_cast<int>(row0));
           pending[c] = true;
         }
@@ -353,8 +355,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       tc_fence_after();
 #pragma unroll 1
       for (int c = 0; c < nch; ++c) {
-        uint32_t r[32];
-        tmem_ld32(tmem_base + (static_cast<uint32_t>(q * 32) << 16) + acc * BN + 32 * c, r);
+        uint32_t r[RES_COLS];
+        tmem_ld16(tmem_base + (static_cast<uint32_t>(q * 32) << 16) + acc * BN + RES_COLS * c, r);
         tmem_wait_ld();
         const int sl = c & 1;
         const bool wh = mbar_wait(&hbar[sl], hph[sl], abort_flag, g.status, WHERE_GEMM);
@@ -366,10 +368,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         pending[sl] = false;
         float* hs = reinterpret_cast<float*>(wbuf + sl * RES_H_BYTES);
         uint8_t* cs = wbuf + 2 * RES_H_BYTES + sl * RES_C_BYTES;
-        float hv[32];
+        float hv[RES_COLS];
 #pragma unroll
-        for (int k = 0; k < 8; ++k) {
-          float4* a = reinterpret_cast<float4*>(hs + lane * 32 + 4 * (k ^ (lane & 7)));
+        for (int k = 0; k < 4; ++k) {
+          // 64-byte rows, 64-byte swizzle: 16-byte chunk k of row r sits at k ^ ((r >> 1) & 3)
+          float4* a = reinterpret_cast<float4*>(hs + lane * 16 + 4 * (k ^ ((lane >> 1) & 3)));
           float4 x = *a;
           x.x += __uint_as_float(r[4 * k]);
           x.y += __uint_as_float(r[4 * k + 1]);
@@ -380,22 +383,23 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         }
         if (copy) {
 #pragma unroll
-          for (int k = 0; k < 4; ++k)
-            *reinterpret_cast<uint4*>(cs + lane * 64 + 16 * (k ^ ((lane >> 1) & 3))) =
+          for (int k = 0; k < 2; ++k)
+            // 32-byte rows, 32-byte swizzle: chunk k of row r sits at k ^ ((r >> 2) & 1)
+            *reinterpret_cast<uint4*>(cs + lane * 32 + 16 * (k ^ ((lane >> 2) & 1))) =
                 make_uint4(pack_bf16x2(hv[8 * k], hv[8 * k + 1]), pack_bf16x2(hv[8 * k + 2], hv[8 * k + 3]),
                            pack_bf16x2(hv[8 * k + 4], hv[8 * k + 5]), pack_bf16x2(hv[8 * k + 6], hv[8 * k + 7]));
         }
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) {
-          const int x = static_cast<int>(colT + 32 * c), y = static_cast<int>(row0);
+          const int x = static_cast<int>(colT + RES_COLS * c), y = static_cast<int>(row0);
           tma_store_2d(&map_h, hs, x, y);
           if (copy) tma_store_2d(&map_c, cs, x, y);
           tma_store_commit();
           if (c + 2 < nch) {
             tma_store_wait_read0();  // the slot's stores have read it
             mbar_arrive_expect_tx(&hbar[sl], RES_H_BYTES);
-            tma_load_2d(&map_h, &hbar[sl], hs, x + 64, y);
+            tma_load_2d(&map_h, &hbar[sl], hs, x + 2 * RES_COLS, y);
             pending[sl] = true;
           }
         }
@@ -485,24 +489,25 @@ cudaError_t gemm_bf16(const GemmArgs& g, cudaStream_t s) {
   const int group = static_cast<int>(std::max<int64_t>(
       1, std::min<int64_t>(m_tiles, clusters / std::min<int64_t>(4, n_tiles))));
   if (g.epi == EPI_STORE) return launch<EPI_STORE>(ma, mb, mb2, ma, ma, g, 2 * clusters, group, s);
-  // residual epilogue: h (fp32, 32x32 boxes, 128-byte swizzle) and its bf16
-  // copy (32x32 boxes, 64-byte swizzle); without a copy the h map stands in
+  // residual epilogue: h (fp32, 16-column x 32-row boxes, 64-byte swizzle) and
+  // its bf16 copy (16 x 32 boxes, 32-byte swizzle); without a copy the h map
+  // stands in
   CUtensorMap mh, mc;
   {
     const uint64_t dims[2] = {static_cast<uint64_t>(g.N), static_cast<uint64_t>(g.M)};
     const uint64_t strides[1] = {static_cast<uint64_t>(g.ldh) * 4};
-    const uint32_t box[2] = {32, 32};
+    const uint32_t box[2] = {RES_COLS, 32};
     if (!encode_tmap(&mh, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, g.h, dims, strides, box,
-                     CU_TENSOR_MAP_SWIZZLE_128B))
+                     CU_TENSOR_MAP_SWIZZLE_64B))
       return cudaErrorInvalidValue;
   }
   mc = mh;
   if (g.h_copy != nullptr) {
     const uint64_t dims[2] = {static_cast<uint64_t>(g.N), static_cast<uint64_t>(g.M)};
     const uint64_t strides[1] = {static_cast<uint64_t>(g.ldhc) * 2};
-    const uint32_t box[2] = {32, 32};
+    const uint32_t box[2] = {RES_COLS, 32};
     if (!encode_tmap(&mc, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, g.h_copy, dims, strides, box,
-                     CU_TENSOR_MAP_SWIZZLE_64B))
+                     CU_TENSOR_MAP_SWIZZLE_32B))
       return cudaErrorInvalidValue;
   }
   return launch<EPI_RESIDUAL>(ma, mb, mb2, mh, mc, g, 2 * clusters, group, s);

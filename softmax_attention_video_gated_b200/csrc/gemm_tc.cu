@@ -13,12 +13,14 @@
 //   warp 1      allocates 512 TMEM columns (pair allocation); on rank 0 one
 //               lane issues M=256 N=256 K=16 MMAs into one of two 256-column
 //               accumulators and multicasts its commits to both CTAs;
-//   warps 2..5  epilogue of this CTA's 128 rows: tcgen05.ld, then a transpose
-//               through shared memory so global reads and writes are
-//               row-contiguous; either a bf16 store (ReLU on leading columns,
-//               the feature map phi of the linear layers) or the residual
-//               update h += C (fp32) with an optional bf16 copy of h. Each warp
-//               releases the accumulator on rank 0's barrier.
+//   warps 2..5  epilogue of this CTA's 128 rows: tcgen05.ld, then either a bf16
+//               store (ReLU on leading columns, the feature map phi of the
+//               linear layers) through a swizzled slot and a TMA store per
+//               32 x 32 chunk, or the residual update h += C (fp32) with an
+//               optional bf16 copy of h. The main loop's TMA writes and MMA
+//               operand reads already take about 128 bytes per clock of shared
+//               memory, so the epilogues keep their own shared-memory traffic
+//               low. Each warp releases the accumulator on rank 0's barrier.
 // A k-block is 128 deep (two boxes per operand) in a 3-stage ring. Every
 // k-block costs the MMA thread one barrier wait and one commit, and those
 // stall its queue of MMAs, so 8 MMAs per k-block run faster than 4: the 720p
@@ -44,9 +46,9 @@ constexpr int HALF = 128;                          // rows of A (and of B) per C
 constexpr int KBOX = HALF * 64 * 2;                // one 128 x 64 bf16 box: 16 KB
 constexpr int TMEM_COLS = 2 * BN;                  // two fp32 accumulators
 constexpr int NUM_THREADS = 192;
-// EPI_STORE epilogue: a 32 x 32 fp32 transpose buffer per warp
-constexpr int STG_STRIDE = 36;                     // fp32 words per staged row (16-byte aligned)
-constexpr int STG_WARP_BYTES = 32 * STG_STRIDE * 4;
+// EPI_STORE epilogue: per warp two slots of a 32 x 32 bf16 chunk (64-byte swizzle)
+constexpr int STO_SLOT_BYTES = 32 * 32 * 2;
+constexpr int STO_WARP_BYTES = 2 * STO_SLOT_BYTES;
 // EPI_RESIDUAL epilogue: per warp two slots of a 32-row x 16-column fp32 chunk
 // of h (64-byte swizzle) and two of its bf16 copy (32-byte swizzle)
 constexpr int RES_COLS = 16;                       // columns of h per chunk
@@ -61,7 +63,7 @@ struct Layout {
   static constexpr int STAGE_BYTES = 2 * A_STAGE;              // A and B, per CTA
   static constexpr int EPI_OFF = STAGES * STAGE_BYTES;
   static_assert(STAGES <= MAX_STAGES, "barrier arrays hold every stage");
-  static constexpr int TAIL_OFF = EPI_OFF + 4 * (EPI == EPI_STORE ? STG_WARP_BYTES : RES_WARP_BYTES);
+  static constexpr int TAIL_OFF = EPI_OFF + 4 * (EPI == EPI_STORE ? STO_WARP_BYTES : RES_WARP_BYTES);
 };
 
 struct GemmTail {
@@ -78,6 +80,11 @@ struct GemmTail {
 template <int EPI>
 constexpr size_t gemm_smem() {
   return 1024 + Layout<EPI>::TAIL_OFF + sizeof(GemmTail);
+}
+
+// bulk stores: wait until at most one committed group still reads shared memory
+__device__ __forceinline__ void tma_store_wait_read1() {
+  asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
 }
 
 __device__ __forceinline__ bool drain_wait(uint64_t* bar, uint32_t parity) {
@@ -151,10 +158,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     tma_prefetch_desc(&map_a);
     tma_prefetch_desc(&map_b);
     if (g.b2 != nullptr) tma_prefetch_desc(&map_b2);
-    if (EPI == EPI_RESIDUAL) {
-      tma_prefetch_desc(&map_h);
-      tma_prefetch_desc(&map_c);
-    }
+    if (EPI == EPI_RESIDUAL) tma_prefetch_desc(&map_h);
+    tma_prefetch_desc(&map_c);
   }
   tc_fence_before();
   cluster_sync();  // both CTAs' barriers exist before either signals the other's
@@ -253,11 +258,15 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     }
   } else if (EPI == EPI_STORE) {
     // ------------------------------------------------ epilogue (warps 2..5, both CTAs)
+    // The thread owning a row packs 32 accumulator columns to bf16 (ReLU on the
+    // leading relu_cols columns) into a 64-byte-swizzled slot, and one TMA
+    // store per 32 x 32 chunk writes them out (TMA clips rows past M and
+    // columns past N). Shared memory sees 2 KB written and 2 KB read per chunk.
     const int q = warp & 3;  // TMEM lane quadrant of this warp
-    float* stg = reinterpret_cast<float*>(smem + Layout<EPI>::EPI_OFF + q * STG_WARP_BYTES);
+    uint8_t* slots = smem + Layout<EPI>::EPI_OFF + q * STO_WARP_BYTES;
     const uint32_t acc_empty0[2] = {cluster_map(&tl->acc_empty[0], 0),
                                     cluster_map(&tl->acc_empty[1], 0)};
-    int local = 0;
+    int local = 0, sl = 0;
     for (int tile = cluster; tile < num_tiles; tile += n_clusters, ++local) {
       const int acc = local & 1;
       const uint32_t acc_phase = (local >> 1) & 1;
@@ -274,44 +283,36 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         tmem_wait_ld();
         const int64_t col0 = static_cast<int64_t>(n_blk) * BN + cc;
         if (col0 >= g.N || row0 >= g.M) continue;  // warp-uniform
-        // stage the warp's 32 rows x 32 columns (thread = row), then read back
-        // four rows per instruction, eight threads per 128-byte row
+        // the store that used this slot two chunks ago has read it
+        if (lane == 0) tma_store_wait_read1();
+        __syncwarp();
+        uint8_t* so = slots + sl * STO_SLOT_BYTES;
+        uint32_t pk[16];
 #pragma unroll
-        for (int k = 0; k < 8; ++k)
-          *reinterpret_cast<uint4*>(stg + lane * STG_STRIDE + 4 * k) =
-              make_uint4(r[4 * k], r[4 * k + 1], r[4 * k + 2], r[4 * k + 3]);
-        __syncwarp();
-        const int sub = lane >> 3, c4 = (lane & 7) * 4;
-        const int64_t col = col0 + c4;
-        const bool col_ok = col + 4 <= g.N;
-#pragma unroll 2
-        for (int it = 0; it < 8; ++it) {
-          const int rr = it * 4 + sub;
-          const int64_t row = row0 + rr;
-          float4 v = *reinterpret_cast<const float4*>(stg + rr * STG_STRIDE + c4);
-          if (row < g.M) {
-            {
-              if (col + 0 < g.relu_cols) v.x = relu_f(v.x);
-              if (col + 1 < g.relu_cols) v.y = relu_f(v.y);
-              if (col + 2 < g.relu_cols) v.z = relu_f(v.z);
-              if (col + 3 < g.relu_cols) v.w = relu_f(v.w);
-              __nv_bfloat16* out = static_cast<__nv_bfloat16*>(g.c) + row * g.ldc + col;
-              if (col_ok) {
-                *reinterpret_cast<uint2*>(out) =
-                    make_uint2(pack_bf16x2(v.x, v.y), pack_bf16x2(v.z, v.w));
-              } else {
-                const float vv[4] = {v.x, v.y, v.z, v.w};
-                for (int e = 0; e < 4 && col + e < g.N; ++e) out[e] = __float2bfloat16_rn(vv[e]);
-              }
-            }
-          }
+        for (int k = 0; k < 16; ++k) {
+          float a = __uint_as_float(r[2 * k]), bb = __uint_as_float(r[2 * k + 1]);
+          if (col0 + 2 * k < g.relu_cols) a = relu_f(a);
+          if (col0 + 2 * k + 1 < g.relu_cols) bb = relu_f(bb);
+          pk[k] = pack_bf16x2(a, bb);
         }
+#pragma unroll
+        for (int k = 0; k < 4; ++k)
+          // 64-byte rows, 64-byte swizzle: chunk k of row r sits at k ^ ((r >> 1) & 3)
+          *reinterpret_cast<uint4*>(so + lane * 64 + 16 * (k ^ ((lane >> 1) & 3))) =
+              make_uint4(pk[4 * k], pk[4 * k + 1], pk[4 * k + 2], pk[4 * k + 3]);
+        fence_proxy_async_smem();
         __syncwarp();
+        if (lane == 0) {
+          tma_store_2d(&map_c, so, static_cast<int>(col0), static_cast<int>(row0));
+          tma_store_commit();
+        }
+        sl ^= 1;
       }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive_cluster(acc_empty0[acc]);
     }
+    if (lane == 0) tma_store_wait0();
   } else {
     // ------------------------------------------------ residual epilogue (warps 2..5, both CTAs)
     // h += C for this warp's 32 rows, 16 columns at a time: TMA brings the h
@@ -488,7 +489,17 @@ cudaError_t gemm_bf16(const GemmArgs& g, cudaStream_t s) {
   // a wave of clusters covers `group` M tiles by about four N tiles
   const int group = static_cast<int>(std::max<int64_t>(
       1, std::min<int64_t>(m_tiles, clusters / std::min<int64_t>(4, n_tiles))));
-  if (g.epi == EPI_STORE) return launch<EPI_STORE>(ma, mb, mb2, ma, ma, g, 2 * clusters, group, s);
+  if (g.epi == EPI_STORE) {
+    // bf16 output C [M, N] in 32 x 32 boxes with a 64-byte swizzle
+    CUtensorMap mo;
+    const uint64_t dims[2] = {static_cast<uint64_t>(g.N), static_cast<uint64_t>(g.M)};
+    const uint64_t strides[1] = {static_cast<uint64_t>(g.ldc) * 2};
+    const uint32_t box[2] = {32, 32};
+    if (!encode_tmap(&mo, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, g.c, dims, strides, box,
+                     CU_TENSOR_MAP_SWIZZLE_64B))
+      return cudaErrorInvalidValue;
+    return launch<EPI_STORE>(ma, mb, mb2, ma, mo, g, 2 * clusters, group, s);
+  }
   // residual epilogue: h (fp32, 16-column x 32-row boxes, 64-byte swizzle) and
   // its bf16 copy (16 x 32 boxes, 32-byte swizzle); without a copy the h map
   // stands in

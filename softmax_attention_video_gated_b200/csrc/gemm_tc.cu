@@ -5,8 +5,8 @@
 // Persistent kernel on clusters of two CTAs (one CTA per SM). A cluster owns
 // 256 x 256 output tiles; the pair shares each tcgen05.mma (cta_group::2):
 // CTA r loads rows [128r, 128r+128) of the A tile and rows [128r, 128r+128) of
-// the B tile (its half of N), so a k-block costs each CTA 32 KB of shared
-// memory instead of the 48 KB a single-CTA 128 x 256 tile needs. Per CTA:
+// the B tile (its half of N), so a 128-deep k-block costs each CTA 64 KB of
+// shared memory instead of the 96 KB a single-CTA 128 x 256 tile needs. Per CTA:
 //   warp 0      TMA producer: 128-row A and B boxes of 64 columns (128-byte
 //               swizzle) into a ring of k-blocks; completion is counted on the
 //               rank-0 CTA's barrier, which expects both CTAs' bytes;

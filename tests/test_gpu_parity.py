@@ -44,7 +44,8 @@ def test_bounded_wait_times_out_and_context_survives():
 # ------------------------------------------------------------------ projections
 
 @pytest.mark.parametrize("dtype", ["bf16", "f32"])
-@pytest.mark.parametrize("M,K,N", [(1, 64, 64), (300, 256, 512), (1000, 512, 320), (517, 192, 1024)])
+@pytest.mark.parametrize("M,K,N", [(1, 64, 64), (300, 256, 512), (1000, 512, 320), (517, 192, 1024),
+                                   (301, 136, 72), (64, 64, 40)])
 def test_projection(dtype, M, K, N):
     rng = np.random.default_rng(M * 7 + N)
     x = W.round_to(rng.standard_normal((M, K)).astype(np.float32), dtype)
@@ -69,9 +70,10 @@ def test_projection_relu_columns(dtype):
 
 
 @pytest.mark.parametrize("dtype", ["bf16", "f32"])
-def test_projection_residual(dtype):
-    rng = np.random.default_rng(4)
-    M, K, N = 333, 256, 512
+@pytest.mark.parametrize("M,K,N", [(333, 256, 512), (77, 136, 200)])
+def test_projection_residual(dtype, M, K, N):
+    # (77, 136, 200): the last N tile ends inside a 16-column chunk of h
+    rng = np.random.default_rng(4 + N)
     x = W.round_to(rng.standard_normal((M, K)).astype(np.float32), dtype)
     w = W.round_to((rng.standard_normal((N, K)) / 16).astype(np.float32), dtype)
     h0 = rng.standard_normal((M, N)).astype(np.float32)

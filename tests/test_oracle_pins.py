@@ -55,6 +55,20 @@ def test_golden_write_gated_linear(golden):
     np.testing.assert_allclose(a[0], c["expect"], rtol=0, atol=1e-14)
 
 
+def test_golden_linear_layer_residual_is_added_after_the_gate(golden):
+    c = golden["linear_layer_residual"]
+    y = O.linear_attn(np.array([c["q"]]), np.array([c["k"]]), np.array([c["v"]]),
+                      np.array([c["g"]]), H=1, eps=c["eps"], residual=np.array([c["residual"]]))
+    np.testing.assert_allclose(y[0], c["expect"], rtol=0, atol=1e-14)
+
+
+def test_golden_softmax_layer_residual_is_added_after_the_gate(golden):
+    c = golden["softmax_layer_residual"]
+    y = O.softmax_anchor(np.array([c["q"]]), np.array([c["k"]]), np.array([c["v"]]),
+                         np.array([c["g"]]), H=1, residual=np.array([c["residual"]]))
+    np.testing.assert_allclose(y[0], c["expect"], rtol=0, atol=1e-14)
+
+
 def test_golden_route(golden):
     c = golden["route"]
     h = np.array([c["h"]])

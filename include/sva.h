@@ -135,8 +135,10 @@ sva_status_t sva_linear_attn_readout_fwd(const sva_attn_args* args, const float*
  * file-scope device array held by every GPU that loads the library until
  * exit; calls needing more return SVA_ERR_WORKSPACE before launching
  * anything. The first call on a device looks up the array's address (make it
- * before any stream capture). All calls on a device share the array: calls
- * that overlap on the GPU race and must be serialised by the caller.
+ * before any stream capture); the address is kept with the device's current
+ * context, and the first call after a device reset (a new context) looks it
+ * up again. All calls on a device share the array: calls that overlap on the
+ * GPU race and must be serialised by the caller.
  * Device-side timeouts are not reported by this entry point.
  */
 sva_status_t sva_linear_attn_fwd_noalloc(const sva_attn_args* args, sva_stream_t stream);
@@ -259,7 +261,7 @@ typedef struct {
   int* prof_count;             /* optional host int                              */
   const void* const* w_wg;     /* optional, L pointers, each [H, D] in dtype     */
   int* launch_count;           /* optional host int: kernels the call launched
-                                  (counted while profiling, prof_events set)    */
+                                  (counted with or without prof_events)         */
 } sva_stack_desc;
 
 size_t sva_hybrid_stack_workspace_bytes(const sva_stack_desc* desc);

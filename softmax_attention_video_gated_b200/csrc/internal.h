@@ -44,6 +44,13 @@ struct ProfScope {
 };
 
 // ---------------------------------------------------------------- utilities
+// Records the CUDA error's text for sva_last_cuda_error and returns SVA_ERR_CUDA.
+sva_status_t cuda_fail(cudaError_t e);
+// Host-side validation of an attention call (null and misaligned pointers,
+// row strides, sizes, eps / scale, supported head sizes). need_kv: k, v (and
+// the write gate) are read; need_qgo: q, gate, out (and the residual) are used.
+sva_status_t check_attn(const sva_attn_args* a, bool linear, bool need_kv = true,
+                        bool need_qgo = true);
 int device_sm_count();
 int device_index();
 bool encode_tmap(CUtensorMap* map, CUtensorMapDataType dt, int rank, const void* base,

@@ -24,12 +24,6 @@ namespace {
 thread_local char g_last_cuda_error[256] = "";
 std::atomic<int> g_sm_count[64];
 
-sva_status_t cuda_fail(cudaError_t e) {
-  snprintf(g_last_cuda_error, sizeof(g_last_cuda_error), "%s: %s", cudaGetErrorName(e),
-           cudaGetErrorString(e));
-  return SVA_ERR_CUDA;
-}
-
 PFN_cuTensorMapEncodeTiled_v12000 get_encode_fn() {
   static std::atomic<void*> fn{nullptr};
   void* p = fn.load();
@@ -49,6 +43,12 @@ bool ld_ok(int64_t ld, int64_t width, sva_dtype_t dt) {
   return ld >= width && (static_cast<size_t>(ld) * esize(dt)) % 16 == 0;
 }
 }  // namespace
+
+sva_status_t cuda_fail(cudaError_t e) {
+  snprintf(g_last_cuda_error, sizeof(g_last_cuda_error), "%s: %s", cudaGetErrorName(e),
+           cudaGetErrorString(e));
+  return SVA_ERR_CUDA;
+}
 
 int device_index() {
   int d = 0;
@@ -91,13 +91,10 @@ using namespace sva;
 // validation
 // ---------------------------------------------------------------------------
 
-namespace {
-
 // need_kv: k, v (and the write gate) are read; need_qgo: q, gate, out (and the
 // residual) are used. The fused calls need both; the two linear-attention
 // phases one each.
-sva_status_t check_attn(const sva_attn_args* a, bool linear, bool need_kv = true,
-                        bool need_qgo = true) {
+sva_status_t sva::check_attn(const sva_attn_args* a, bool linear, bool need_kv, bool need_qgo) {
   if (a == nullptr) return SVA_ERR_INVALID_ARGUMENT;
   if (a->dtype != SVA_F32 && a->dtype != SVA_BF16) return SVA_ERR_INVALID_ARGUMENT;
   if (a->B < 1 || a->N < 1 || a->H < 1 || a->d < 1) return SVA_ERR_INVALID_ARGUMENT;
@@ -123,6 +120,8 @@ sva_status_t check_attn(const sva_attn_args* a, bool linear, bool need_kv = true
   if (a->dtype == SVA_F32 && a->d != 64 && a->d != 128) return SVA_ERR_UNSUPPORTED;
   return SVA_OK;
 }
+
+namespace {
 
 sva_status_t clear_status(void* ws, cudaStream_t s) {
   cudaError_t e = cudaMemsetAsync(ws, 0, SVA_STATUS_BYTES, s);
@@ -452,12 +451,16 @@ sva_status_t stack_pass(const sva_stack_desc* desc, const void* x, void* y, void
   if (ws == nullptr || !aligned16(ws) || ws_bytes < lay.total) return SVA_ERR_WORKSPACE;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
 
+  // launches are counted whenever the caller asks for the count; events are
+  // recorded only when it hands some over
   Prof prof_obj;
   Prof* prof = nullptr;
-  if (d.prof_events != nullptr) {
-    prof_obj.events = reinterpret_cast<cudaEvent_t*>(const_cast<void**>(d.prof_events));
-    prof_obj.capacity = d.prof_capacity;
-    prof_obj.kinds = d.prof_kind;
+  if (d.prof_events != nullptr || d.launch_count != nullptr) {
+    if (d.prof_events != nullptr) {
+      prof_obj.events = reinterpret_cast<cudaEvent_t*>(const_cast<void**>(d.prof_events));
+      prof_obj.capacity = d.prof_capacity;
+      prof_obj.kinds = d.prof_kind;
+    }
     prof = &prof_obj;
   }
 

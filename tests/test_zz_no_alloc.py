@@ -20,8 +20,8 @@ if not torch.cuda.is_available():
 import softmax_attention_video_gated_b200 as sva  # noqa: E402
 
 
-def noalloc_call(q, k, v, g, out, H, eps=1e-6):
-    a = sva._attn_args(q, k, v, g, out, H, None, eps, 0.0, 0)
+def noalloc_call(q, k, v, g, out, H, eps=1e-6, residual=None, wgate=None):
+    a = sva._attn_args(q, k, v, g, out, H, residual, eps, 0.0, 0, wgate)
     return sva._lib().sva_linear_attn_fwd_noalloc(ctypes.byref(a), sva._stream())
 
 
@@ -38,6 +38,26 @@ def test_noalloc_matches_workspace_entry_point_on_two_calls_in_a_row(dtype):
         assert noalloc_call(t["q"], t["k"], t["v"], t["g"], out, H) == sva.SVA_OK
         torch.cuda.synchronize()
         assert_close(to_host(out), to_host(ref), dtype, f"noalloc B={B} N={N}")
+
+
+def test_noalloc_with_residual_and_write_gate_matches_workspace_entry_point():
+    # the residual and write-gate operands go through the same validation and
+    # kernels as in the workspace entry point; out aliases the residual
+    B, N, H = 1, 2333, 2
+    x = W.core_inputs(B, N, H, 128, "bf16", 103)
+    t = {k: to_dev(v, "bf16") for k, v in x.items()}
+    wg = to_dev(W.normal((B, N, H), 1.0, 103, W.TAG_WGATE, "bf16"), "bf16")
+    # a residual of the layer output's own scale (~0.05), so neither term hides the other
+    r = to_dev(W.normal((B, N, H * 128), 0.05, 104, W.TAG_X, "bf16"), "bf16")
+    for _ in range(2):
+        ref = r.clone()
+        sva.sva_linear_attn_fwd(t["q"], t["k"], t["v"], t["g"], ref, H, residual=ref, eps=1e-6,
+                                wgate=wg)
+        out = r.clone()
+        assert noalloc_call(t["q"], t["k"], t["v"], t["g"], out, H, residual=out,
+                            wgate=wg) == sva.SVA_OK
+        torch.cuda.synchronize()
+        assert_close(to_host(out), to_host(ref), "bf16", "noalloc residual + write gate")
 
 
 def test_noalloc_refuses_calls_beyond_its_scratch():

@@ -409,6 +409,11 @@ class Stack:
         self.desc.prof_count = ctypes.pointer(self.prof_count)
         self.desc.launch_count = ctypes.pointer(self.launch_count)
 
+    def count_launches(self):
+        """Have each later call write the number of kernels it launched to
+        self.launch_count (no events recorded)."""
+        self.desc.launch_count = ctypes.pointer(self.launch_count)
+
     def clear_profile(self):
         self.desc.prof_events = None
         self.desc.prof_capacity = 0

@@ -47,7 +47,7 @@ closed forms, library routines, invariants); none is "parity unpinned".
 from __future__ import annotations
 
 import math
-from typing import Dict, List, Optional, Sequence, Tuple
+from typing import Callable, Dict, List, Optional, Sequence, Tuple
 
 import numpy as np
 
@@ -260,7 +260,8 @@ def block_of(l: int, attnres_block: int) -> int:
 
 def stack(x, w_qkvg: Sequence[np.ndarray], w_o: Sequence[np.ndarray], w_r, H: int,
           softmax_period: int = 4, attnres_block: int = 8, all_softmax: bool = False,
-          eps: float = 1e-6, keep_trace: bool = False, w_wg: Optional[Sequence] = None):
+          eps: float = 1e-6, keep_trace: bool = False, w_wg: Optional[Sequence] = None,
+          on_layer: Optional[Callable] = None):
     """The hybrid token mixer: tokens in, mixed tokens out.
 
     h_0 = x; for l = 1..L: u = routed or plain input, [Q|K|V|G] = u W_qkvg[l]^T,
@@ -271,7 +272,10 @@ def stack(x, w_qkvg: Sequence[np.ndarray], w_o: Sequence[np.ndarray], w_r, H: in
     write-gated, the logits being W = u W_wg[l]^T.
 
     Returns y = h_L and, when keep_trace, a dict of per-layer lists
-    u, Y, o (each [B, N, D]) and alpha ([B, N, c-1] or None), plus kinds."""
+    u, Y, o (each [B, N, D]) and alpha ([B, N, c-1] or None), plus kinds.
+    on_layer, if given, is called after each layer as
+    on_layer(l, kind, u, Y, o, alpha) (an observer: it changes nothing), so a
+    caller can inspect every layer of a stack too large to keep whole."""
     h = _f64(x).copy()
     D = h.shape[-1]
     L = len(w_qkvg)
@@ -296,6 +300,8 @@ def stack(x, w_qkvg: Sequence[np.ndarray], w_o: Sequence[np.ndarray], w_r, H: in
         h = h + o
         if attnres_block > 0 and l % attnres_block == 0:
             summaries.append(h.copy())
+        if on_layer is not None:
+            on_layer(l, kind, u, Y, o, alpha)
         if keep_trace:
             trace["u"].append(u)
             trace["Y"].append(Y)

@@ -2,9 +2,12 @@
 times (one call per layer over all heads): attention outputs are checked on
 sampled query rows the oracle computes one by one against all keys (tile
 edges, the pair boundary of the anchor's two-tile CTAs and the ragged tail
-included); the 8-layer 480p stack is checked whole; the 24-layer 720p stack,
-too large for the fp64 oracle, is checked through properties that hold at any
-size (token-permutation equivariance, run-to-run determinism).
+included); the 8-layer 480p stack is checked whole; the 24-layer 720p stack
+is also checked through properties that hold at any
+size (token-permutation equivariance, run-to-run determinism); the oracle's
+whole-stack comparison of the 720p stack is in test_gpu_stacks_whole.py. The
+anchor is also checked at the duration sweep's longest lengths (N = 148,120
+and 221,720).
 
 Inputs up to 720p come from the chunked numpy generator; the linear sweep's
 largest lengths (1.9 GB per tensor) are drawn by torch's seeded generator on
@@ -94,6 +97,33 @@ def test_long_video_layers_sampled_rows():
     rows = sample_rows(w.N, seed=1)
     for kind in ("anchor", "linear"):
         check_rows(kind, x, run_core(kind, t, w.H), w.H, rows)
+
+
+# ------------------------------------------------------------------ anchor at long-video lengths
+
+@pytest.mark.parametrize("N", [148120, 221720])
+def test_anchor_long_duration_sampled_rows(N):
+    # the softmax anchor at 161 and 241 latent frames of 23 x 40 patches (the
+    # 40 s and 60 s rows of the duration sweep), one call over all 24 heads, as
+    # the sweep times it; inputs drawn on the device, K and V copied to the host
+    # in bf16 and handed to the oracle one head at a time (heads are independent)
+    H, d, seed = 24, 128, 1234 + 5
+    D = H * d
+    t = {name: W.normal_torch((1, N, D), 1.0, seed, tag, "bf16")
+         for name, tag in (("q", W.TAG_Q), ("k", W.TAG_K), ("v", W.TAG_V), ("g", W.TAG_G))}
+    out = run_core("anchor", t, H)
+    rows = sample_rows(N, seed=N)
+    ri = torch.as_tensor(rows, device="cuda")
+    q, g = to_host(t["q"][:, ri]), to_host(t["g"][:, ri])
+    got = to_host(out[:, ri])
+    k_h, v_h = t["k"].cpu(), t["v"].cpu()
+    del t, out
+    ref = np.empty_like(got)
+    for h in range(H):
+        c = slice(h * d, (h + 1) * d)
+        ref[..., c] = O.softmax_anchor(q[..., c], k_h[..., c].to(torch.float64).numpy(),
+                                       v_h[..., c].to(torch.float64).numpy(), g[..., c], 1)
+    assert_close(got, ref, "bf16", f"anchor sampled rows N={N}")
 
 
 # ------------------------------------------------------------------ linear sweep (B = 2)

@@ -384,6 +384,26 @@ def test_stack_batch_entries_are_independent():
                                    rtol=1e-13, atol=1e-14)
 
 
+def test_stack_layer_observer_sees_the_traced_layers_and_changes_nothing():
+    # on_layer is an observer: the result is unchanged, and it sees exactly the
+    # per-layer values keep_trace records
+    x, wq, wo, wr, H = small_stack(L=12)
+    y, tr = O.stack(x, wq, wo, wr, H, keep_trace=True)
+    seen = []
+    y2 = O.stack(x, wq, wo, wr, H, on_layer=lambda *a: seen.append(a))
+    np.testing.assert_array_equal(y2, y)
+    assert [a[0] for a in seen] == list(range(1, 13))
+    for l, kind, u, Y, o, alpha in seen:
+        assert kind == tr["kind"][l - 1]
+        np.testing.assert_array_equal(u, tr["u"][l - 1])
+        np.testing.assert_array_equal(Y, tr["Y"][l - 1])
+        np.testing.assert_array_equal(o, tr["o"][l - 1])
+        if alpha is None:
+            assert tr["alpha"][l - 1] is None
+        else:
+            np.testing.assert_array_equal(alpha, tr["alpha"][l - 1])
+
+
 def test_stack_zero_output_projection_is_identity():
     x, wq, wo, wr, H = small_stack(L=12, wo_zero=True)
     np.testing.assert_array_equal(O.stack(x, wq, wo, wr, H), x)

@@ -219,8 +219,8 @@ def stack_x(w: StackWorkload) -> np.ndarray:
 def normal_torch(shape, std: float, seed: int, tag: int, dtype: str, device="cuda"):
     """N(0, std^2) drawn by torch's seeded Philox generator on `device`, rounded
     to `dtype` (torch's round-to-nearest-even). Used where numpy would take
-    minutes (the 720p stack's 1.1e9 weights); tensors drawn here are never
-    compared element by element with the oracle."""
+    minutes (the 720p stack's 1.1e9 weights, the long-video activations); the
+    tests copy such tensors to the host to give the oracle their exact values."""
     import torch
     g = torch.Generator(device=device)
     g.manual_seed((seed * 1000003 + tag) & 0x7FFFFFFFFFFFFFFF)

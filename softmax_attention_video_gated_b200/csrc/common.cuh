@@ -100,6 +100,30 @@ __device__ __forceinline__ uint64_t add_f2(uint64_t a, uint64_t b) {
   asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
   return r;
 }
+// Integer hash of a 32-bit counter (xor-shift / multiply rounds; the
+// constants are Chris Wellons' "lowbias32" from his published hash survey).
+__device__ __forceinline__ uint32_t hash32(uint32_t x) {
+  x ^= x >> 16;
+  x *= 0x7feb352du;
+  x ^= x >> 15;
+  x *= 0x846ca68bu;
+  x ^= x >> 16;
+  return x;
+}
+
+// Two fp32 values to bf16 with unbiased (stochastic) rounding: 16 random bits
+// are added below each value's bf16 precision before the low 16 bits are cut,
+// so a value rounds away from zero with probability equal to the fraction of
+// the bf16 step it holds and E[bf16(x)] = x. Round-to-nearest is biased where
+// a value is a bf16 number plus less than half a step (that small part is
+// always lost); unbiased rounding keeps it on average over many values.
+// rnd: low 16 bits dither lo, high 16 bits dither hi. Finite inputs only.
+__device__ __forceinline__ uint32_t pack_bf16x2_unbiased(float lo, float hi, uint32_t rnd) {
+  const uint32_t a = __float_as_uint(lo) + (rnd & 0xFFFFu);
+  const uint32_t b = __float_as_uint(hi) + (rnd >> 16);
+  return (a >> 16) | (b & 0xFFFF0000u);
+}
+
 __device__ __forceinline__ float max3_f(float a, float b, float c) {
   float r;
   asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));

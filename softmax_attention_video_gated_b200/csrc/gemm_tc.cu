@@ -383,12 +383,24 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           hv[4 * k] = x.x; hv[4 * k + 1] = x.y; hv[4 * k + 2] = x.z; hv[4 * k + 3] = x.w;
         }
         if (copy) {
+          uint32_t pk[RES_COLS / 2];
+          if (g.copy_dither != 0u) {
+            // one hash per column pair of this row: (seed, row, pair) -> 32 bits
+            const uint32_t rkey = g.copy_dither ^ (static_cast<uint32_t>(row0 + lane) * 0x9E3779B1u);
+            const uint32_t pair0 = static_cast<uint32_t>((colT + RES_COLS * c) >> 1);
+#pragma unroll
+            for (int k = 0; k < RES_COLS / 2; ++k)
+              pk[k] = pack_bf16x2_unbiased(hv[2 * k], hv[2 * k + 1],
+                                           hash32(rkey + (pair0 + k) * 0x85EBCA77u));
+          } else {
+#pragma unroll
+            for (int k = 0; k < RES_COLS / 2; ++k) pk[k] = pack_bf16x2(hv[2 * k], hv[2 * k + 1]);
+          }
 #pragma unroll
           for (int k = 0; k < 2; ++k)
             // 32-byte rows, 32-byte swizzle: chunk k of row r sits at k ^ ((r >> 2) & 1)
             *reinterpret_cast<uint4*>(cs + lane * 32 + 16 * (k ^ ((lane >> 2) & 1))) =
-                make_uint4(pack_bf16x2(hv[8 * k], hv[8 * k + 1]), pack_bf16x2(hv[8 * k + 2], hv[8 * k + 3]),
-                           pack_bf16x2(hv[8 * k + 4], hv[8 * k + 5]), pack_bf16x2(hv[8 * k + 6], hv[8 * k + 7]));
+                make_uint4(pk[4 * k], pk[4 * k + 1], pk[4 * k + 2], pk[4 * k + 3]);
         }
         fence_proxy_async_smem();
         __syncwarp();

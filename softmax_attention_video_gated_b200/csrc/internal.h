@@ -75,6 +75,10 @@ struct GemmArgs {
   int relu_cols = 0;
   float* h = nullptr;       int64_t ldh = 0;   // EPI_RESIDUAL: fp32 stream
   void* h_copy = nullptr;   int64_t ldhc = 0;  // EPI_RESIDUAL: optional copy
+  // EPI_RESIDUAL, bf16: 0 = the copy is rounded to nearest; otherwise it is
+  // rounded without bias (pack_bf16x2_unbiased), the random bits hashed from
+  // this seed, the row and the column pair (deterministic)
+  uint32_t copy_dither = 0;
   int* status = nullptr;
 };
 

@@ -81,15 +81,19 @@ def _whole_stack_parity(w):
     update = to_host(update).reshape(B, N, D)
 
     checked = []
+    worst = {"Y": 0.0, "o": 0.0, "alpha": 0.0}
 
     def on_layer(l, kind, u, Y, o, alpha):
         i = l - 1
-        assert_close(to_host(trace_y[i]).reshape(Y.shape), Y, "bf16", f"Y_{l} ({kind})")
-        assert_close(to_host(trace_o[i]).reshape(o.shape), o, "bf16", f"o_{l} ({kind})")
+        r = assert_close(to_host(trace_y[i]).reshape(Y.shape), Y, "bf16", f"Y_{l} ({kind})")
+        worst["Y"] = max(worst["Y"], r)
+        r = assert_close(to_host(trace_o[i]).reshape(o.shape), o, "bf16", f"o_{l} ({kind})")
+        worst["o"] = max(worst["o"], r)
         if nb[i]:
             assert alpha is not None and alpha.shape[-1] == nb[i]
-            assert_close(to_host(trace_alpha[i]).reshape(alpha.shape), alpha, "bf16",
-                         f"alpha_{l} ({nb[i]} blocks)")
+            r = assert_close(to_host(trace_alpha[i]).reshape(alpha.shape), alpha, "bf16",
+                             f"alpha_{l} ({nb[i]} blocks)")
+            worst["alpha"] = max(worst["alpha"], r)
         else:
             assert alpha is None
         checked.append((l, kind, nb[i]))
@@ -99,8 +103,9 @@ def _whole_stack_parity(w):
                    to_host(wr), w.H, softmax_period=w.softmax_period,
                    attnres_block=w.attnres_block, on_layer=on_layer)
     assert [c[0] for c in checked] == list(range(1, L + 1))
-    assert_close(update, yref - xh, "bf16", "h_L - x")
-    assert_close(to_host(y), yref, "bf16", "y")
+    worst["h_L - x"] = assert_close(update, yref - xh, "bf16", "h_L - x")
+    worst["y"] = assert_close(to_host(y), yref, "bf16", "y")
+    print(f"{w.name}: worst rel-L2 " + ", ".join(f"{k} {v:.2e}" for k, v in worst.items()))
     return checked
 
 

@@ -112,7 +112,8 @@ sva_status_t sva_linear_attn_fwd(const sva_attn_args* args, void* ws, size_t ws_
  * shards, summed (an all-reduce), are the state of the whole sequence, and
  * each shard's queries then read it out. The state is fp32, per (batch,
  * head) d*d + d values: S row-major (row = d_k, column = d_v), then z; size it
- * with sva_linear_attn_state_bytes (1.58 MB for B = 1, H = 24, d = 128).
+ * with sva_linear_attn_state_bytes (1.58 MB for B = 1, H = 24, d = 128); it
+ * must be 16-byte aligned.
  *   sva_linear_attn_state_fwd:   uses k, v (and wgate) of args->N tokens and
  *                                writes the state; q, gate, out are ignored.
  *   sva_linear_attn_readout_fwd: uses q, gate, out (and residual) of args->N

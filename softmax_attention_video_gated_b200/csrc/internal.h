@@ -89,7 +89,7 @@ cudaError_t transpose_2d(const void* src, void* dst, int64_t rows, int64_t cols,
 
 // ---------------------------------------------------------------- linear attention
 // Scratch of one linear-attention call (offsets from the scratch base):
-// fp32 per-chunk partial states, then the reduced state.
+// fp32 per-chunk partial states, then (fp32 path only) the reduced state.
 struct LinearPlan {
   int tiles_per_chunk = 0;  // 128-token tiles per state chunk (bf16) / tokens per chunk (f32)
   int n_chunks = 0;

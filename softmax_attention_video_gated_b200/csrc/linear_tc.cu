@@ -8,22 +8,26 @@
 // sigmoid(W_t), one logit per token and head (same section: the gate sets how
 // much each token writes into the state).
 //
-// Three kernels, all HBM-bound (the roofline is 10 B*N*D bytes of Q, K, V, G
+// Two kernels, both HBM-bound (the roofline is 10 B*N*D bytes of Q, K, V, G
 // and Y traffic per layer):
 //  1. lin_state_tc:  one CTA per (token chunk, head, batch). TMA streams
 //     128-token K and V tiles into a 3-stage ring; four warps apply ReLU in
 //     shared memory and accumulate z; one thread issues tcgen05.mma with
 //     A = phi(K)^T and B = V, both read MN-major straight from the TMA layout,
-//     accumulating the 128x128 fp32 partial state in TMEM.
-//  2. lin_reduce: sums the chunk partials in chunk order (deterministic) and
-//     writes the read-out operand [S^T | z_hi | z_lo | 0] as bf16 [144 x 128]
-//     (z split in two bf16 rows keeps it to ~16 bits).
-//  3. lin_readout_tc: persistent over the same chunks as the state pass. The
-//     state operand is loaded once; Q and G tiles stream through a 2-stage
-//     TMA ring; one M=128, N=144, K=128 MMA per tile gives the numerator
-//     (columns 0..127) and denominator (columns 128, 129) together into one of
-//     two TMEM accumulators; eight epilogue warps divide, apply the sigmoid
-//     gate and residual, and write Y through per-warp TMA stores.
+//     accumulating the 128x128 fp32 partial state of the chunk in TMEM, which
+//     goes to global memory (66 KB per chunk, read back from L2).
+//  2. lin_readout_tc: persistent over the same chunks as the state pass. Its
+//     epilogue warps first sum the head's chunk partials in chunk order
+//     (deterministic, the same in every CTA of the head) into the read-out
+//     operand [S^T | z_hi | z_lo | 0], bf16 [144 x 128] in shared memory (z
+//     split in two bf16 rows keeps it to ~16 bits), while the first Q and G
+//     tiles land. Q and G tiles stream through a 2-stage TMA ring; one M=128,
+//     N=144, K=128 MMA per tile gives the numerator (columns 0..127) and
+//     denominator (columns 128, 129) together into one of two TMEM
+//     accumulators; eight epilogue warps divide, apply the sigmoid gate and
+//     residual, and write Y through per-warp TMA stores.
+//  Summing the partials in the read-out instead of a separate kernel removes
+//  one launch and one kernel boundary per layer.
 #include <algorithm>
 
 #include "common.cuh"
@@ -284,67 +288,9 @@ __global__ void __launch_bounds__(192, 1)
   }
 }
 
-// ------------------------------------------------------------------ reduce
-// state_op[bh] = bf16 [144][128]: rows 0..127 = S^T (row n = d_v, column k =
-// d_k), row 128 = bf16(z), row 129 = bf16(z - bf16(z)), rows 130..143 = 0.
-// One CTA per 32x32 tile of S (16 per head): sums the chunk partials in chunk
-// order (deterministic) and writes the tile transposed through shared memory.
-__global__ void __launch_bounds__(256) lin_reduce_bf16_kernel(const float* __restrict__ partial,
-                                                              __nv_bfloat16* __restrict__ state_op,
-                                                              int n_chunks) {
-  __shared__ float tile[32][33];
-  const int64_t bh = blockIdx.y;
-  const int ki = blockIdx.x >> 2, ni = blockIdx.x & 3;
-  const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;
-  const int elems = HD * HD + HD;
-  const float* p = partial + bh * n_chunks * elems;
-  __nv_bfloat16* o = state_op + bh * STATE_ROWS * HD;
-  if (n_chunks <= 8) {
-    // all 4 x n_chunks loads issued before any add (latency, not bandwidth, bounds this)
-    float v[4][8];
-#pragma unroll
-    for (int r = 0; r < 4; ++r) {
-      const float* pp = p + (ki * 32 + ty + 8 * r) * HD + ni * 32 + tx;
-#pragma unroll
-      for (int c = 0; c < 8; ++c) v[r][c] = c < n_chunks ? pp[static_cast<int64_t>(c) * elems] : 0.f;
-    }
-#pragma unroll
-    for (int r = 0; r < 4; ++r) {
-      float acc = 0.f;
-#pragma unroll
-      for (int c = 0; c < 8; ++c) acc += v[r][c];
-      tile[ty + 8 * r][tx] = acc;
-    }
-  } else {
-#pragma unroll
-    for (int r = 0; r < 4; ++r) {
-      const int k = ki * 32 + ty + 8 * r, n = ni * 32 + tx;
-      float acc = 0.f;
-      for (int c = 0; c < n_chunks; ++c) acc += p[static_cast<int64_t>(c) * elems + k * HD + n];
-      tile[ty + 8 * r][tx] = acc;
-    }
-  }
-  __syncthreads();
-#pragma unroll
-  for (int r = 0; r < 4; ++r) {
-    const int n = ni * 32 + ty + 8 * r, k = ki * 32 + tx;
-    o[n * HD + k] = __float2bfloat16_rn(tile[tx][ty + 8 * r]);
-  }
-  if (blockIdx.x == 0) {
-    for (int e = threadIdx.x; e < HD; e += 256) {
-      float acc = 0.f;
-      for (int c = 0; c < n_chunks; ++c) acc += p[static_cast<int64_t>(c) * elems + HD * HD + e];
-      const __nv_bfloat16 hi = __float2bfloat16_rn(acc);
-      o[HD * HD + e] = hi;
-      o[(HD + 1) * HD + e] = __float2bfloat16_rn(acc - __bfloat162float(hi));
-    }
-    for (int e = threadIdx.x; e < (STATE_ROWS - HD - 2) * HD; e += 256)
-      o[(HD + 2) * HD + e] = __float2bfloat16_rn(0.f);
-  }
-}
-
+// ------------------------------------------------------------------ state only
 // fp32 state of one (batch, head), [S (d_k rows x d_v) | z]: the chunk partials
-// summed in chunk order (the same order as the fused path's reduce)
+// summed in chunk order (the same order as the read-out's own sum)
 __global__ void __launch_bounds__(256) lin_sum_chunks_kernel(const float* __restrict__ partial,
                                                              float* __restrict__ state,
                                                              int n_chunks) {
@@ -361,7 +307,8 @@ __global__ void __launch_bounds__(256) lin_sum_chunks_kernel(const float* __rest
 // ------------------------------------------------------------------ read-out
 // Persistent over the state pass's chunks (one CTA per (token chunk, head,
 // batch), one wave). The head's read-out operand [S^T | z_hi | z_lo | 0] is
-// loaded once; 128-token tiles of Q and G stream through a 2-stage TMA ring.
+// built once (build_state_operand); 128-token tiles of Q and G stream through
+// a 2-stage TMA ring.
 // One M=128, N=144, K=128 MMA per tile gives numerator (columns 0..127) and
 // denominator (128, 129) into one of two TMEM accumulators, so the MMA of the
 // next tile runs during this tile's epilogue. Eight epilogue warps: warp w
@@ -393,11 +340,100 @@ struct ReadoutTail {
 constexpr size_t kReadoutSmem = 1024 + RO_TAIL_OFF + sizeof(ReadoutTail);
 constexpr int RO_TMEM_COLS = 512;                      // two 256-column accumulators
 
+// The read-out operand of head (b, h), built by the 256 epilogue threads
+// straight into shared memory: [S^T | z_hi | z_lo | 0] as bf16 [144 x 128],
+// K-major in two [64-column x 144-row] boxes with the 128-byte swizzle the MMA
+// descriptor expects (16-byte chunk c of row r at chunk c ^ (r & 7)). S and z
+// are the sums of the n_chunks fp32 partial states in chunk order (the same
+// order for every CTA of the head, so they all build the same operand). The
+// partials (66 KB each) are read from L2 with float4 loads: thread t sums
+// columns n = 4 (t % 32) .. +3 of S (rows of S^T) over k in two 8-wide groups
+// (t / 32 and t / 32 + 8).
+__device__ __forceinline__ void build_state_operand(const float* __restrict__ part, int n_chunks,
+                                                    uint8_t* op, int et) {
+  constexpr int ELEMS = HD * HD + HD;
+  const int nq = et & 31, kset = et >> 5;
+  float acc[2][8][4];
+#pragma unroll
+  for (int g = 0; g < 2; ++g)
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) acc[g][i][e] = 0.f;
+#pragma unroll 1
+  for (int c = 0; c < n_chunks; ++c) {
+    const float* pc = part + static_cast<int64_t>(c) * ELEMS + 4 * nq;
+    float4 v[2][8];
+#pragma unroll
+    for (int g = 0; g < 2; ++g)
+#pragma unroll
+      for (int i = 0; i < 8; ++i)
+        v[g][i] = *reinterpret_cast<const float4*>(pc + (8 * (kset + 8 * g) + i) * HD);
+#pragma unroll
+    for (int g = 0; g < 2; ++g)
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        acc[g][i][0] += v[g][i].x;
+        acc[g][i][1] += v[g][i].y;
+        acc[g][i][2] += v[g][i].z;
+        acc[g][i][3] += v[g][i].w;
+      }
+  }
+  // row n of S^T, k-group kg: 8 bf16 = one 16-byte chunk
+#pragma unroll
+  for (int g = 0; g < 2; ++g) {
+    const int kg = kset + 8 * g;  // k = 8 kg .. 8 kg + 7
+    uint8_t* box = op + (kg >> 3) * STATE_BOX_BYTES;
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const int n = 4 * nq + e;
+      uint4 o;
+      o.x = pack_bf16x2(acc[g][0][e], acc[g][1][e]);
+      o.y = pack_bf16x2(acc[g][2][e], acc[g][3][e]);
+      o.z = pack_bf16x2(acc[g][4][e], acc[g][5][e]);
+      o.w = pack_bf16x2(acc[g][6][e], acc[g][7][e]);
+      *reinterpret_cast<uint4*>(box + n * 128 + (((kg & 7) ^ (n & 7)) << 4)) = o;
+    }
+  }
+  // rows 128, 129: z split into a bf16 head and its bf16 remainder; rows 130..143: 0
+  if (et < 16) {
+    const int kg = et;
+    float z[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) z[i] = 0.f;
+#pragma unroll 1
+    for (int c = 0; c < n_chunks; ++c) {
+      const float4* pz =
+          reinterpret_cast<const float4*>(part + static_cast<int64_t>(c) * ELEMS + HD * HD + 8 * kg);
+      const float4 a = pz[0], b = pz[1];
+      z[0] += a.x; z[1] += a.y; z[2] += a.z; z[3] += a.w;
+      z[4] += b.x; z[5] += b.y; z[6] += b.z; z[7] += b.w;
+    }
+    uint32_t hi[4], lo[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      hi[i] = pack_bf16x2(z[2 * i], z[2 * i + 1]);
+      lo[i] = pack_bf16x2(z[2 * i] - bf16lo_to_f32(hi[i]), z[2 * i + 1] - bf16hi_to_f32(hi[i]));
+    }
+    uint8_t* box = op + (kg >> 3) * STATE_BOX_BYTES;
+    *reinterpret_cast<uint4*>(box + HD * 128 + (((kg & 7) ^ (HD & 7)) << 4)) =
+        make_uint4(hi[0], hi[1], hi[2], hi[3]);
+    *reinterpret_cast<uint4*>(box + (HD + 1) * 128 + (((kg & 7) ^ ((HD + 1) & 7)) << 4)) =
+        make_uint4(lo[0], lo[1], lo[2], lo[3]);
+  }
+  for (int i = et; i < 2 * (STATE_ROWS - HD - 2) * 8; i += 256) {
+    const int bx = i / ((STATE_ROWS - HD - 2) * 8), rem = i % ((STATE_ROWS - HD - 2) * 8);
+    const int r = HD + 2 + rem / 8, ch = rem % 8;
+    *reinterpret_cast<uint4*>(op + bx * STATE_BOX_BYTES + r * 128 + (ch << 4)) =
+        make_uint4(0u, 0u, 0u, 0u);
+  }
+}
+
 __global__ void __launch_bounds__(RO_THREADS, 1)
     lin_readout_tc_kernel(const __grid_constant__ CUtensorMap map_q,
                           const __grid_constant__ CUtensorMap map_g,
-                          const __grid_constant__ CUtensorMap map_s,
-                          const __grid_constant__ CUtensorMap map_o, int N, int H,
+                          const __grid_constant__ CUtensorMap map_o,
+                          const float* __restrict__ partial, int n_chunks, int N, int H,
                           int tiles_per_chunk, float eps, unsigned flags,
                           const __nv_bfloat16* residual, int64_t ldr, int* status) {
   extern __shared__ uint8_t smem_raw[];
@@ -421,7 +457,7 @@ __global__ void __launch_bounds__(RO_THREADS, 1)
       mbar_init(&tl->acc_full[a], 1);
       mbar_init(&tl->acc_empty[a], 8);
     }
-    mbar_init(&tl->s_full, 1);
+    mbar_init(&tl->s_full, 8);  // one arrival per epilogue warp once the operand is built
     mbar_init(&tl->drain, 1);
     tl->abort_flag = 0;
     fence_mbar_init();
@@ -439,10 +475,6 @@ __global__ void __launch_bounds__(RO_THREADS, 1)
   if (warp == 0) {
     if (lane == 0 && ntiles > 0) {
       // ------------------------------------------------ TMA producer
-      const int srow = (b * H + h) * STATE_ROWS;
-      mbar_arrive_expect_tx(&tl->s_full, 2 * STATE_BOX_BYTES);
-      tma_load_2d(&map_s, &tl->s_full, smem + RO_S_OFF, 0, srow);
-      tma_load_2d(&map_s, &tl->s_full, smem + RO_S_OFF + STATE_BOX_BYTES, 64, srow);
       int stage = 0;
       uint32_t phase = 0;
       int issued = 0;
@@ -465,7 +497,6 @@ __global__ void __launch_bounds__(RO_THREADS, 1)
           phase ^= 1;
         }
       }
-      (void)drain_wait(&tl->s_full, 0);
       if (!ok)
         for (int i = max(0, issued - RO_STAGES); i < issued; ++i)
           (void)drain_wait(&tl->full[i % RO_STAGES], (i / RO_STAGES) & 1);
@@ -515,6 +546,12 @@ __global__ void __launch_bounds__(RO_THREADS, 1)
     const int r = wq * 32 + lane;            // row of the tile
     const uint32_t lane_base = static_cast<uint32_t>(wq * 32) << 16;
     uint8_t* yslot = smem + RO_Y_OFF + ew * RO_Y_SLOT;
+    // the head's read-out operand, while the producer's first Q and G tiles land
+    build_state_operand(partial + static_cast<int64_t>(b * H + h) * n_chunks * (HD * HD + HD),
+                        n_chunks, smem + RO_S_OFF, threadIdx.x - 64);
+    fence_proxy_async_smem();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&tl->s_full);
     // ReLU on this thread's half-row of Q in tile k (its stage), then report it
     auto relu_tile = [&](int k) -> bool {
       const int st = k % RO_STAGES;
@@ -654,8 +691,8 @@ LinearPlan linear_plan(int B, int N, int H, int d, sva_dtype_t dt) {
   const size_t elems = static_cast<size_t>(d) * d + d;
   p.partial_off = 0;
   p.state_off = align_up(p.partial_off + static_cast<size_t>(p.n_chunks) * work * elems * 4, 1024);
-  const size_t state_bytes = dt == SVA_BF16 ? static_cast<size_t>(work) * STATE_ROWS * HD * 2
-                                            : static_cast<size_t>(work) * elems * 4;
+  // bf16: the read-out builds its operand in shared memory; fp32: the reduced state
+  const size_t state_bytes = dt == SVA_BF16 ? 0 : static_cast<size_t>(work) * elems * 4;
   p.total = align_up(p.state_off + state_bytes, 1024);
   return p;
 }
@@ -665,7 +702,6 @@ cudaError_t linear_bf16(const sva_attn_args& a, int* status, void* scratch, cuda
   const LinearPlan p = linear_plan(a.B, a.N, a.H, a.d, SVA_BF16);
   char* base = static_cast<char*>(scratch);
   float* partial = reinterpret_cast<float*>(base + p.partial_off);
-  __nv_bfloat16* state = reinterpret_cast<__nv_bfloat16*>(base + p.state_off);
   const int D = a.H * a.d;
   cudaError_t e;
   if (state_in == nullptr) {
@@ -686,23 +722,20 @@ cudaError_t linear_bf16(const sva_attn_args& a, int* status, void* scratch, cuda
                                          a.ldw, partial, status);
       if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
-    ProfScope ps(prof, s, SVA_KERNEL_LINEAR_REDUCE);
     if (state_out != nullptr) {
       // state only: the fp32 state, for the caller to sum over token shards
+      ProfScope ps(prof, s, SVA_KERNEL_LINEAR_REDUCE);
       lin_sum_chunks_kernel<<<dim3((HD * HD + HD + 255) / 256, a.B * a.H), 256, 0, s>>>(
           partial, state_out, p.n_chunks);
       return cudaGetLastError();
     }
-    lin_reduce_bf16_kernel<<<dim3(16, a.B * a.H), 256, 0, s>>>(partial, state, p.n_chunks);
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  } else {
-    // read-out of a given fp32 state: its read-out operand, as from one chunk
-    ProfScope ps(prof, s, SVA_KERNEL_LINEAR_REDUCE);
-    lin_reduce_bf16_kernel<<<dim3(16, a.B * a.H), 256, 0, s>>>(state_in, state, 1);
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
   // ------------------------------------------------ read-out (Q, G, Y of these tokens)
-  CUtensorMap mq, mg, mo, ms;
+  // Each read-out CTA sums its head's partial states itself (or takes a given
+  // fp32 state, as one chunk) into the bf16 read-out operand in shared memory.
+  const float* parts = state_in != nullptr ? state_in : partial;
+  const int n_parts = state_in != nullptr ? 1 : p.n_chunks;
+  CUtensorMap mq, mg, mo;
   if (!act_map(&mq, a.q, a.ldq, a.B, a.N, D) || !act_map(&mg, a.gate, a.ldg, a.B, a.N, D))
     return cudaErrorInvalidValue;
   {
@@ -716,20 +749,12 @@ cudaError_t linear_bf16(const sva_attn_args& a, int* status, void* scratch, cuda
                      CU_TENSOR_MAP_SWIZZLE_128B))
       return cudaErrorInvalidValue;
   }
-  {
-    const uint64_t dims[2] = {HD, static_cast<uint64_t>(a.B) * a.H * STATE_ROWS};
-    const uint64_t strides[1] = {HD * 2};
-    const uint32_t box[2] = {64, STATE_ROWS};
-    if (!encode_tmap(&ms, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, state, dims, strides, box,
-                     CU_TENSOR_MAP_SWIZZLE_128B))
-      return cudaErrorInvalidValue;
-  }
   ProfScope ps(prof, s, SVA_KERNEL_LINEAR_READOUT);
   e = cudaFuncSetAttribute(lin_readout_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            static_cast<int>(kReadoutSmem));
   if (e != cudaSuccess) return e;
   lin_readout_tc_kernel<<<dim3(p.n_chunks, a.H, a.B), RO_THREADS, kReadoutSmem, s>>>(
-      mq, mg, ms, mo, a.N, a.H, p.tiles_per_chunk, a.eps, a.flags,
+      mq, mg, mo, parts, n_parts, a.N, a.H, p.tiles_per_chunk, a.eps, a.flags,
       static_cast<const __nv_bfloat16*>(a.residual), a.ldr, status);
   return cudaGetLastError();
 }

@@ -26,8 +26,8 @@
 // by more than 8 (p <= 2^8 otherwise, exact after the final 1/l); the max uses
 // three-input max, and the scale-and-shift and the row sum run on packed fp32
 // pairs (one f32x2 FFMA or FADD per two keys). Exponentials run on the MUFU
-// unit; kPolyEvery can send every k-th one to the FMA pipe instead (Cody-Waite
-// reduction and a minimax cubic, see fit_exp2_poly.py).
+// unit (sending a share of them to the FMA pipe as a polynomial was measured
+// slower: the MUFU pipe is not what bounds this kernel).
 // What bounds it (720p layer on B200, clock64 traces of one CTA, ncu): each
 // tile's chain -- softmax of block j (about 2,100 cycles, 1,260 of them on the
 // exponentials), then P_j V_j and S_{j+1} on the tensor core (about 1,250),
@@ -64,12 +64,6 @@ constexpr float kRescaleThreshold = 8.0f;    // log2 units
 // register split: 128 threads at 56 + 256 threads at 224 = 384 threads at 168
 constexpr int kRegsProducer = 56, kRegsSoftmax = 224;
 
-// every kPolyEvery-th exponential of a row is evaluated on the FMA pipe (0: none)
-constexpr int kPolyEvery = 0;
-// minimax cubic for 2^f on [-1/2, 1/2] with c0 = 1 (fit_exp2_poly.py);
-// max relative error 4.4e-4, five times below bf16's rounding of P
-constexpr float kP1 = 0.695766806602478f, kP2 = 0.24203051626682281f, kP3 = 0.041698750108480453f;
-
 struct AnchorTail {
   uint64_t q_full;
   uint64_t k_full[K_STAGES];
@@ -94,27 +88,6 @@ __device__ __forceinline__ float ex2_mufu(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
-}
-
-// 2^x on the FMA pipe: x = n + f with n = rint(x) (1.5 * 2^23 added and taken
-// away), 2^f by the cubic, 2^n by adding n to the exponent bits. x is clamped at
-// -127, where the result is exactly 0 (n = -127, f = 0).
-__device__ __forceinline__ float ex2_poly(float x) {
-  x = fmaxf(x, -127.0f);
-  const float t = x + 12582912.0f;
-  const float f = x - (t - 12582912.0f);
-  const float p = fmaf(fmaf(fmaf(kP3, f, kP2), f, kP1), f, 1.0f);
-  // the low bits of t hold n; the bits of 1.5 * 2^23 shifted by 23 vanish mod 2^32
-  return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
-}
-
-// exponential of the element at position `idx` of a row
-template <int kEvery>
-__device__ __forceinline__ float ex2_row(float x, int idx) {
-  if constexpr (kEvery > 0) {
-    if (idx % kEvery == kEvery - 1) return ex2_poly(x);
-  }
-  return ex2_mufu(x);
 }
 
 // Work of one launch: units (query-tile pair, head, batch), x fastest. The
@@ -390,8 +363,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             float x0, x1;
             f2unpack(fma_f2(f2pack(s[32 * c + 2 * i], s[32 * c + 2 * i + 1]), scale2, negm2), x0,
                      x1);
-            const float p0 = ex2_row<kPolyEvery>(x0, 2 * i);
-            const float p1 = ex2_row<kPolyEvery>(x1, 2 * i + 1);
+            const float p0 = ex2_mufu(x0);
+            const float p1 = ex2_mufu(x1);
             acc2[i & 3] = add_f2(acc2[i & 3], f2pack(p0, p1));
             pk[i] = pack_bf16x2(p0, p1);
           }

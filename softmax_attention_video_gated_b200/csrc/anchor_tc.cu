@@ -15,7 +15,10 @@
 //        gate G into Q's buffer, so the epilogue reads G from shared memory
 //        (it used to wait on DRAM for each 32-column chunk: ~17,000 cycles of
 //        a CTA's ~560,000 with the tensor pipe idle; 720p 3.87 -> 3.79 ms);
-//        warp 2: TMA for the V tiles (2-stage ring). K is released as
+//        warp 2: TMA for the V tiles (2-stage ring); warp 3: checks that V_j and
+//        K_{j+1} have landed and adds one arrival to each tile's P barrier, so
+//        the MMA thread waits on P only and the softmax reports P without that
+//        check on its chain (720p 3.75 -> 3.69-3.72 ms). K is released as
 //        soon as both S MMAs of a block have read it, V after both P V MMAs,
 //        so the next block's K is already resident when its S MMA is due.
 //        warp 1: allocates all 512 TMEM columns (tile t: S_t at 256t, O_t at
@@ -47,7 +50,8 @@
 // shared-memory descriptors are therefore built once and offset by constants
 // (8,190 keys: 0.87 -> 0.79 ms; 720p: 3.94 -> 3.90 ms). Earlier steps:
 // packed pairs 4.35 -> 4.02 ms; the waits for V_j and K_{j+1} moved from the
-// MMA thread to a softmax warp of each tile, 3.94 ms.
+// MMA thread to a softmax warp of each tile, 3.94 ms; later to warp 3, with
+// warp-uniform role loops and G prefetched for the epilogue: 3.69-3.72 ms.
 #include <algorithm>
 #include <math.h>
 
@@ -153,7 +157,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&tl->s_full[i], 1);
-      mbar_init(&tl->p_full[i], 128);
+      mbar_init(&tl->p_full[i], 129);  // + warp 3: V_j, K_{j+1} resident
     }
     mbar_init(&tl->o_done, 1);
     mbar_init(&tl->g_full, 1);
@@ -262,6 +266,27 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         for (int i = max(0, issued - V_STAGES); i < issued; ++i)
           (void)drain_wait(&tl->v_full[i % V_STAGES], (i / V_STAGES) & 1);
       __syncwarp();
+    } else if (warp == 3) {
+      // ------------------------------------------------ residency of V_j and K_{j+1}
+      // one arrival per tile and block on p_full once both have landed; it
+      // waits for that phase to complete before checking the next block, so
+      // it never arrives twice in one phase
+      const int ntiles = has1 ? 2 : 1;
+      for (int j = 0; j < nkv; ++j) {
+        bool w = mbar_wait(&tl->v_full[j % V_STAGES], (j / V_STAGES) & 1, abort_flag, status,
+                           WHERE_ANCHOR);
+        if (j + 1 < nkv)
+          w = w && mbar_wait(&tl->k_full[(j + 1) % K_STAGES], ((j + 1) / K_STAGES) & 1, abort_flag,
+                             status, WHERE_ANCHOR);
+        if (!__all_sync(0xffffffffu, w)) break;
+        if (lane == 0)
+          for (int t = 0; t < ntiles; ++t) mbar_arrive(&tl->p_full[t]);
+        __syncwarp();
+        bool wp = true;
+        for (int t = 0; t < ntiles; ++t)
+          wp = wp && mbar_wait(&tl->p_full[t], j & 1, abort_flag, status, WHERE_ANCHOR);
+        if (!__all_sync(0xffffffffu, wp)) break;
+      }
     } else if (warp == 1) {
       // ------------------------------------------------ MMA issuer
       constexpr uint32_t idesc_s = idesc_bf16_f32(BQ, BKV, false, false);  // Q, K: K-major
@@ -310,8 +335,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       int vst = 0, kn = 1 % K_STAGES;  // stages of V_j and K_{j+1}
       for (int j = 0; j < nkv && ok; ++j) {
         const bool more = j + 1 < nkv;
-        // V_j and K_{j+1} need no wait here: a softmax warp of each tile saw
-        // them land before it reported P_j (its p_full arrival orders them)
+        // V_j and K_{j+1} need no wait here: warp 3 saw them land before its
+        // arrival on p_full, which the P_j wait below includes
         for (int t = 0; t < ntiles; ++t) {
           const bool w = mbar_wait(&tl->p_full[t], j & 1, abort_flag, status, WHERE_ANCHOR);
           if (!__all_sync(0xffffffffu, w)) {
@@ -435,20 +460,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           l += u0 + u1;
         }
         tc_fence_before();
-        if (q == 0) {
-          // the MMA thread waits only for P: this warp checks that V_j and
-          // K_{j+1} are resident before P_j is reported (it has slack; the MMA
-          // thread's waits are on the critical path)
-          bool w = mbar_wait(&tl->v_full[j % V_STAGES], (j / V_STAGES) & 1, abort_flag, status,
-                             WHERE_ANCHOR);
-          if (j + 1 < nkv)
-            w = w && mbar_wait(&tl->k_full[(j + 1) % K_STAGES], ((j + 1) / K_STAGES) & 1,
-                               abort_flag, status, WHERE_ANCHOR);
-          if (!__all_sync(0xffffffffu, w)) {
-            ok = false;
-            break;
-          }
-        }
         mbar_arrive(&tl->p_full[t]);
       }
       if (ok && nkv > 0) {

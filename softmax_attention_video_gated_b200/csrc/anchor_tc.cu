@@ -39,19 +39,22 @@
 // unit (sending a share of them to the FMA pipe as a polynomial was measured
 // slower: the MUFU pipe is not what bounds this kernel).
 // What bounds it (720p layer on B200, clock64 traces of one CTA, ncu): each
-// tile's chain -- softmax of block j (about 2,100 cycles, 1,260 of them on the
-// exponentials), then P_j V_j and S_{j+1} on the tensor core (about 1,250),
-// then the wake-ups -- sets the step at about 3,700 cycles for two tiles, and
-// the tensor and MUFU pipes are each active about half of the time. Alone, a
-// 128x128x16 MMA takes its nominal 64 cycles in every form used here (also
-// back to back on aliased columns, and with other warps reading TMEM); inside
-// the kernel the MMA thread shares its SM sub-partition with two busy softmax
-// warps, so its own instruction count sets how fast MMAs are issued: its
-// shared-memory descriptors are therefore built once and offset by constants
-// (8,190 keys: 0.87 -> 0.79 ms; 720p: 3.94 -> 3.90 ms). Earlier steps:
-// packed pairs 4.35 -> 4.02 ms; the waits for V_j and K_{j+1} moved from the
-// MMA thread to a softmax warp of each tile, 3.94 ms; later to warp 3, with
-// warp-uniform role loops and G prefetched for the epilogue: 3.69-3.72 ms.
+// tile's chain -- softmax of block j (about 1,700 cycles: S load 70, block
+// max 350, exponentials and P stores 1,190, report 100), then the MMA warp
+// noticing P (~350), P_j V_j and S_{j+1} on the tensor core (about 1,370; the
+// S MMAs, both operands in shared memory, ~97 cycles each against 64 nominal),
+// then the softmax seeing S_{j+1} (~150) -- sets the step at about 3,580
+// cycles for two tiles. The exponential loop is near its minimum instruction
+// count, and any instruction added to it lengthens it (a polynomial for part
+// of the exponentials, or the block max folded into it). ncu against the
+// library's sm100 flash kernel at the same shape shows the same MMA count and
+// the same shared-memory and TMEM traffic; that kernel runs 16 warps and
+// issues more per cycle. Descriptors are built once and offset by constants,
+// since the MMA warp's own instruction count reaches the tensor pipe (8,190
+// keys: 0.87 -> 0.79 ms; 720p: 3.94 -> 3.90 ms). Earlier steps: packed pairs
+// 4.35 -> 4.02 ms; the waits for V_j and K_{j+1} moved from the MMA thread to
+// a softmax warp of each tile, 3.94 ms; later to warp 3, with warp-uniform
+// role loops and G prefetched for the epilogue: 3.66-3.72 ms.
 #include <algorithm>
 #include <math.h>
 

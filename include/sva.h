@@ -99,7 +99,8 @@ typedef struct {
  *     S = sum_t omega_t phi(K_t)^T V_t,   z = sum_t omega_t phi(K_t).
  * Supported: SVA_BF16 with d = 128 (tcgen05 kernels), SVA_F32 with d in
  * {64, 128}. Any N >= 1. The workspace holds per-chunk partial states (fp32)
- * and the reduced state; size it with sva_linear_attn_workspace_bytes.
+ * and, for SVA_F32, the reduced state (the bf16 read-out sums the partials
+ * itself); size it with sva_linear_attn_workspace_bytes.
  * The softmax anchor ignores wgate.
  */
 size_t sva_linear_attn_workspace_bytes(int B, int N, int H, int d, sva_dtype_t dtype);

@@ -1,13 +1,15 @@
 """The allocation-free linear-attention entry point, for callers that cannot
 allocate device memory (an engine with a fixed memory plan, a plugin handed a
 stream but no allocator): it must give the same results as the workspace entry
-point, call after call, while its scratch lives in the library's fixed device
-array. Collected last so a failure here leaves every other test already run."""
+point and match the fp64 oracle, call after call, while its scratch lives in
+the library's fixed device array. Collected last so a failure here leaves every
+other test already run."""
 import ctypes
 
 import numpy as np
 import pytest
 
+import oracle as O
 import workloads as W
 from tests._util import assert_close, to_dev, to_host
 
@@ -38,6 +40,8 @@ def test_noalloc_matches_workspace_entry_point_on_two_calls_in_a_row(dtype):
         assert noalloc_call(t["q"], t["k"], t["v"], t["g"], out, H) == sva.SVA_OK
         torch.cuda.synchronize()
         assert_close(to_host(out), to_host(ref), dtype, f"noalloc B={B} N={N}")
+        want = O.linear_attn(x["q"], x["k"], x["v"], x["g"], H, eps=1e-6)
+        assert_close(to_host(out), want, dtype, f"noalloc B={B} N={N} vs oracle")
 
 
 def test_noalloc_with_residual_and_write_gate_matches_workspace_entry_point():
@@ -46,9 +50,12 @@ def test_noalloc_with_residual_and_write_gate_matches_workspace_entry_point():
     B, N, H = 1, 2333, 2
     x = W.core_inputs(B, N, H, 128, "bf16", 103)
     t = {k: to_dev(v, "bf16") for k, v in x.items()}
-    wg = to_dev(W.normal((B, N, H), 1.0, 103, W.TAG_WGATE, "bf16"), "bf16")
+    wg_h = W.normal((B, N, H), 1.0, 103, W.TAG_WGATE, "bf16")
+    wg = to_dev(wg_h, "bf16")
     # a residual of the layer output's own scale (~0.05), so neither term hides the other
-    r = to_dev(W.normal((B, N, H * 128), 0.05, 104, W.TAG_X, "bf16"), "bf16")
+    r_h = W.normal((B, N, H * 128), 0.05, 104, W.TAG_X, "bf16")
+    r = to_dev(r_h, "bf16")
+    want = O.linear_attn(x["q"], x["k"], x["v"], x["g"], H, eps=1e-6, residual=r_h, wgate=wg_h)
     for _ in range(2):
         ref = r.clone()
         sva.sva_linear_attn_fwd(t["q"], t["k"], t["v"], t["g"], ref, H, residual=ref, eps=1e-6,
@@ -58,6 +65,7 @@ def test_noalloc_with_residual_and_write_gate_matches_workspace_entry_point():
                             wgate=wg) == sva.SVA_OK
         torch.cuda.synchronize()
         assert_close(to_host(out), to_host(ref), "bf16", "noalloc residual + write gate")
+        assert_close(to_host(out), want, "bf16", "noalloc residual + write gate vs oracle")
 
 
 def test_noalloc_refuses_calls_beyond_its_scratch():

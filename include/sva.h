@@ -154,7 +154,10 @@ sva_status_t sva_linear_attn_fwd_noalloc(const sva_attn_args* args, sva_stream_t
  * and v (n_keys = 0: the same N tokens; otherwise e.g. one shard's queries
  * against the all-gathered keys and values of the whole sequence).
  * No N x N matrix is stored. Supported: SVA_BF16 with d = 128 (tcgen05 flash
- * kernel), SVA_F32 with d in {64, 128}. Workspace: status word only.
+ * kernel), SVA_F32 with d in {64, 128}. Workspace: the status word, and for
+ * SVA_BF16 the last wave's key-split parts (each part's unnormalised O, running
+ * max and row sum, combined by a merge kernel); size it with
+ * sva_softmax_anchor_workspace_bytes, which bounds it over every key count.
  */
 size_t sva_softmax_anchor_workspace_bytes(int B, int N, int H, int d, sva_dtype_t dtype);
 sva_status_t sva_softmax_anchor_fwd(const sva_attn_args* args, void* ws, size_t ws_bytes,

@@ -132,7 +132,7 @@ sva_status_t sva_linear_attn_readout_fwd(const sva_attn_args* args, const float*
  * results) for callers that cannot allocate device memory when they run the
  * mixer: engines that plan all device memory at start-up and allow no
  * allocation afterwards, plugins handed a stream but no allocator, programs
- * whose memory pool belongs to another framework. The paper has no
+ * whose memory pool belongs to another framework. The method has no
  * counterpart; this is a library convenience. The scratch is a 16 MiB
  * file-scope device array held by every GPU that loads the library until
  * exit; calls needing more return SVA_ERR_WORKSPACE before launching
